@@ -1,0 +1,138 @@
+"""Seeded synthetic decode workloads (inputs only -- no attention arithmetic).
+
+Every input of the tests and of the benchmark comes from here, so the CUDA
+path and the fp64 oracle always see the same bits.  Recipe, per workload:
+
+* values are drawn with ``torch.randn`` from a ``torch.Generator`` seeded with
+  ``seed`` on the device the tensors live on, in fp32, in the fixed order
+  q, k, v (k and v in slices of at most ``_SLICE`` elements along the
+  flattened [B*H*N, D] rows), multiplied by ``scale`` and then rounded to the
+  workload's element type;
+* ALiBi slopes are the fp32 values 2^(-8(h+1)/H), h = 0..H-1;
+* ragged lengths are ``torch.randint(lo, hi+1, (B,))`` from a CPU generator
+  seeded with ``seed + 1``; keys at positions >= N_b of the padded [B,H,Nmax,D]
+  buffers are filled like the rest but never read;
+* "peaked" workloads pick, per (b,h), ``spikes`` distinct key positions with
+  ``torch.randperm`` from a CPU generator seeded with ``seed + 2`` and set
+  k_j <- 8 * ||k_j|| * q/||q|| (fp32, before rounding), so those keys score far
+  above the rest.
+
+The five named workloads are the shapes the decode kernel is measured on; any
+field can be overridden (smaller N, B, H) for parity runs the oracle finishes
+in seconds.
+"""
+from dataclasses import dataclass, replace
+from typing import Optional, Tuple
+
+import torch
+
+_SLICE = 1 << 26
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    dtype: torch.dtype
+    B: int
+    H: int
+    D: int
+    N: int                      # keys per sequence (the padded Nmax when ragged)
+    n_split: int = 0            # splits per (b,h); 0 = library heuristic
+    alibi: bool = False
+    ragged: Optional[Tuple[int, int]] = None   # inclusive [lo, hi] of N_b
+    scale: float = 1.0
+    spikes: int = 0
+    seed: int = 1234
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+    @property
+    def elt(self) -> int:
+        return torch.tensor([], dtype=self.dtype).element_size()
+
+
+WORKLOADS = {
+    # gist shape: one head, D=512, 4096 keys, split into 8 chunks, fp32
+    "gist_f32_d512_n4k": Workload("gist_f32_d512_n4k", torch.float32, 1, 1, 512, 4096,
+                                  n_split=8, seed=1234),
+    # long-context bf16 decode, 32 heads, 128K keys, split count automatic
+    "bf16_h32_d128_n128k": Workload("bf16_h32_d128_n128k", torch.bfloat16, 1, 32, 128,
+                                    131072, seed=1235),
+    # batched bf16 decode with the ALiBi broadcast row
+    "bf16_alibi_b8_h32_d128_n32k": Workload("bf16_alibi_b8_h32_d128_n32k", torch.bfloat16,
+                                            8, 32, 128, 32768, alibi=True, seed=1236),
+    # 1M-key bf16 decode with a peaked softmax (16 spiked keys per head)
+    "bf16_peaked_h8_d128_n1m": Workload("bf16_peaked_h8_d128_n1m", torch.bfloat16, 1, 8,
+                                        128, 1 << 20, scale=0.5, spikes=16, seed=1237),
+    # fp16 batched decode, ragged lengths U[1024, 65536], padded to 65536
+    "f16_ragged_b64_h16_d64": Workload("f16_ragged_b64_h16_d64", torch.float16, 64, 16, 64,
+                                       65536, ragged=(1024, 65536), seed=1238),
+}
+
+
+def alibi_slopes(H: int, device="cpu") -> torch.Tensor:
+    """Per-head ALiBi slopes 2^(-8(h+1)/H) as fp32."""
+    h = torch.arange(H, dtype=torch.float64)
+    return torch.pow(2.0, -8.0 * (h + 1) / H).to(torch.float32).to(device)
+
+
+def seqlens_for(w: Workload) -> Optional[torch.Tensor]:
+    if w.ragged is None:
+        return None
+    lo, hi = w.ragged
+    lo = min(lo, w.N)
+    hi = min(hi, w.N)
+    g = torch.Generator(device="cpu").manual_seed(w.seed + 1)
+    return torch.randint(lo, hi + 1, (w.B,), generator=g, dtype=torch.int64).to(torch.int32)
+
+
+def _randn_rows(gen, rows, D, device, scale, dtype):
+    """[rows, D] of N(0,1)*scale in dtype, drawn in fp32 slices."""
+    out = torch.empty((rows, D), dtype=dtype, device=device)
+    step = max(1, _SLICE // D)
+    for r0 in range(0, rows, step):
+        r1 = min(rows, r0 + step)
+        x = torch.randn((r1 - r0, D), generator=gen, device=device, dtype=torch.float32)
+        if scale != 1.0:
+            x.mul_(scale)
+        out[r0:r1].copy_(x)
+    return out
+
+
+def make_inputs(w: Workload, device="cpu"):
+    """Materialise a workload: dict(q, k, v, slopes, seqlens, seqlens_host)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    B, H, D, N = w.B, w.H, w.D, w.N
+    qf = torch.randn((B, H, 1, D), generator=g, device=device, dtype=torch.float32)
+    if w.scale != 1.0:
+        qf.mul_(w.scale)
+    q = qf.to(w.dtype)
+    k = _randn_rows(g, B * H * N, D, device, w.scale, w.dtype).view(B, H, N, D)
+    v = _randn_rows(g, B * H * N, D, device, w.scale, w.dtype).view(B, H, N, D)
+    sl_host = seqlens_for(w)
+    if w.spikes:
+        gs = torch.Generator(device="cpu").manual_seed(w.seed + 2)
+        for b in range(B):
+            n_b = int(sl_host[b]) if sl_host is not None else N
+            for h in range(H):
+                pos = torch.randperm(n_b, generator=gs)[: min(w.spikes, n_b)].to(device)
+                kj = k[b, h, pos].float()
+                qd = qf[b, h, 0] / qf[b, h, 0].norm()
+                k[b, h, pos] = (8.0 * kj.norm(dim=-1, keepdim=True) * qd).to(w.dtype)
+    slopes = alibi_slopes(H, device) if w.alibi else None
+    seqlens = sl_host.to(device) if sl_host is not None else None
+    return dict(q=q, k=k, v=v, slopes=slopes, seqlens=seqlens, seqlens_host=sl_host)
+
+
+def kv_lengths(w: Workload, seqlens_host: Optional[torch.Tensor]) -> int:
+    """Sum over (b,h) of the keys actually attended."""
+    if seqlens_host is None:
+        return w.B * w.H * w.N
+    return int(seqlens_host.to(torch.int64).sum()) * w.H
+
+
+def kv_bytes(w: Workload, seqlens_host: Optional[torch.Tensor]) -> int:
+    """Algorithmic bytes of one decode step: every attended K and V row once."""
+    return 2 * kv_lengths(w, seqlens_host) * w.D * w.elt
