@@ -1,0 +1,440 @@
+"""Benchmark of one decode step of libtreedec on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one td_decode call over the whole workload: the split-KV kernel
+with its fused ticket combine (the entire hot path, one launch).  Inputs are
+seeded synthetic tensors already resident in HBM; the default workload
+(bf16, B=1, H=32, D=128, N=131072) moves 2 GiB of K+V per step, far beyond the
+126 MB L2, so no flush is needed between steps.  Prints one JSON line on
+rank 0.  Under torchrun every rank decodes its own copy of the workload on its
+own GPU (independent problems, weak scaling, no data-path collective).
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0
+only), each step a bounded sample of the same workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from long_context_attention_td_b200.workloads import WORKLOADS, kv_bytes, kv_lengths, make_inputs  # noqa: E402
+
+METRIC = "decode attention KV GB/s and % of B200 HBM peak (1 GPU); µs per decode step"
+DEFAULT_WORKLOAD = "bf16_h32_d128_n128k"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DTYPE_NAME = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float16: "f16"}
+KERNEL_SOURCES = ["td_partial.cu", "td_device.cuh", "td_internal.cuh"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for s in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "long_context_attention_td_b200", "csrc", s), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the split-KV kernel from the committed ncu
+    summary of this workload, or None if absent or taken on other sources."""
+    path = os.path.join(ROOT, "profiles", "td_partial_%s.md" % workload)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", text)
+    m_bytes = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+        return None
+    return int(m_bytes.group(1))
+
+
+# ------------------------------------------------------------------ clocks
+
+_REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+                0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons every 200 ms."""
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            ident = str(device_index)
+        self.ident = ident
+
+    def start(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
+        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, "--query-gpu=" + q,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                bits = int(parts[3], 16)
+            except ValueError:
+                continue
+            for b, n in _REASON_BITS.items():
+                if bits & b and n != "gpu_idle":
+                    reasons.add(n)
+        sm.sort()
+        med = sm[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def reduce_max(x, device):
+    """Max of a float over ranks (x itself when not distributed)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x, device):
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+# -------------------------------------------------------------- CPU oracle
+
+def oracle_rate(inp, w, budget_s, min_s=0.0, threads=0):
+    """Time the fp64 oracle on (b,h) rows of a host copy of the workload;
+    returns (GB/s, threads used, description, seconds)."""
+    import oracle
+    B, H = w.B, w.H
+    cores = os.cpu_count() or 1
+    threads = threads or cores
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    lens = inp["seqlens_host"]
+    per_head = [int(lens[b]) if lens is not None else w.N for b in range(B) for _ in range(H)]
+    # rows to time: one per thread, first (b,h) pairs, shortened so one pass
+    # stays within the budget at ~0.5 GB/s per core
+    n_rows = min(B * H, threads)
+    est_rate = 0.5e9 * n_rows
+    keys_cap = max(1024, int(budget_s * est_rate / (2 * w.D * w.elt * n_rows)))
+    rows = list(range(n_rows))
+    nk = min(max(per_head[r] for r in rows), keys_cap)
+    qs = q.reshape(B * H, 1, 1, w.D)[rows].cpu()
+    ks = k.reshape(B * H, 1, w.N, w.D)[rows, :, :nk].cpu()
+    vs = v.reshape(B * H, 1, w.N, w.D)[rows, :, :nk].cpu()
+    sl = None
+    if lens is not None:
+        sl = torch.tensor([min(per_head[r], nk) for r in rows], dtype=torch.int32)
+    slopes = inp["slopes"]
+    s1 = None if slopes is None else slopes.cpu()[[r % H for r in rows]]
+    bytes_once = sum(2 * (min(per_head[r], nk)) * w.D * w.elt for r in rows)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        if s1 is None:
+            oracle.full(qs.view(len(rows), 1, 1, w.D), ks.view(len(rows), 1, nk, w.D),
+                        vs.view(len(rows), 1, nk, w.D), seqlens=None if sl is None else sl,
+                        threads=threads)
+        else:
+            # per-row slope: rows are independent sequences with H = 1
+            for i in range(len(rows)):
+                oracle.full(qs[i:i + 1], ks[i:i + 1], vs[i:i + 1], slopes=s1[i:i + 1],
+                            seqlens=None if sl is None else sl[i:i + 1], threads=1)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            break
+    rate = bytes_once * passes / dt / 1e9
+    desc = ("%d (b,h) rows x %d keys (%s, D=%d), %d pass(es), %d thread(s)"
+            % (len(rows), nk, DTYPE_NAME[w.dtype], w.D, passes, min(threads, len(rows))))
+    return rate, min(threads, len(rows)), desc, dt
+
+
+# -------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import long_context_attention_td_b200 as td
+
+    world, rank, local = dist_setup(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    inp = make_inputs(w, dev)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    n_split = w.n_split if args.n_split is None else args.n_split
+    stream = torch.cuda.current_stream(dev)
+    B, H, D, N = w.B, w.H, w.D, w.N
+    total_keys = kv_lengths(w, inp["seqlens_host"])
+    parts = td.plan_parts(B, H, N, D, w.dtype, n_split,
+                          total_keys if inp["seqlens"] is not None else -1)
+
+    def step():
+        if inp["seqlens"] is not None:
+            td.decode_varlen(q, k, v, inp["seqlens"], seqlens_host=inp["seqlens_host"],
+                             slopes=inp["slopes"], n_split=n_split, out=out, lse=lse,
+                             stream=stream)
+        else:
+            td.decode(q, k, v, slopes=inp["slopes"], n_split=n_split, out=out, lse=lse,
+                      stream=stream)
+
+    out = torch.empty((B, H, 1, D), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, H, 1), dtype=torch.float32, device=dev)
+    bytes_step = kv_bytes(w, inp["seqlens_host"])
+
+    sampler = ClockSampler(dev.index).start()
+    t_load0 = time.perf_counter()
+    for _ in range(args.warmup):
+        step()
+    td.check_device_error(stream=stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    # keep the GPU loaded until the clock sampler has seen >= 1 s of load
+    while time.perf_counter() - t_load0 < 1.2:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    td.check_device_error(stream=stream)
+
+    # the dominant (only) kernel per step, timed launch by launch on its stream
+    n_kt = min(args.steps, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_kt)]
+    for a, b in evs:
+        a.record(stream)
+        step()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    kernel_ms = sum(a.elapsed_time(b) for a, b in evs) / n_kt
+
+    ms_max = reduce_max(ms_total, dev)
+    bytes_all = reduce_sum(float(bytes_step) * args.steps, dev)
+    kernel_ms_max = reduce_max(kernel_ms, dev)
+    ms_per_step = ms_max / args.steps
+    value = bytes_all / (ms_max * 1e-3) / 1e9
+    per_gpu = bytes_step / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the host-buffer entry point (pinned host inputs)
+    e2e = None
+    if not args.no_e2e:
+        qh = q.cpu().pin_memory()
+        kh = k.cpu().pin_memory()
+        vh = v.cpu().pin_memory()
+        sh = inp["seqlens_host"]
+        slh = None if inp["slopes"] is None else inp["slopes"].cpu()
+        oh = torch.empty((B, H, 1, D), dtype=torch.float32).pin_memory()
+        lh = torch.empty((B, H, 1), dtype=torch.float32).pin_memory()
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+        for _ in range(2):
+            td.decode_host(qh, kh, vh, seqlens=sh, slopes=slh, n_split=n_split, out=oh, lse=lh,
+                           stream=stream, sync=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            td.decode_host(qh, kh, vh, seqlens=sh, slopes=slh, n_split=n_split, out=oh, lse=lh,
+                           stream=stream, sync=False)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = reduce_max(e0.elapsed_time(e1), dev)
+        e_bytes = reduce_sum(float(bytes_step) * e2e_steps, dev)
+        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        h2d += 0 if slh is None else slh.numel() * 4
+        h2d += 0 if sh is None else sh.numel() * 4
+        d2h = oh.numel() * 4 + lh.numel() * 4
+        e2e = {"value": round(e_bytes / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": e2e_steps, "ms_per_step": round(e_ms / e2e_steps, 4),
+               "entry_point": "td_decode_host"}
+        del qh, kh, vh
+
+    peak, peak_kind = measured_peak()
+    achieved = bytes_step / (kernel_ms_max * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+                "traffic": profiled_traffic(args.workload),
+                "kernel": "td_partial_kernel (fused ticket combine)",
+                "algorithmic_bytes_per_launch": int(bytes_step)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, used, desc, dt = oracle_rate(inp, w, budget_s=2.0, min_s=args.cpu_seconds)
+        cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2), "host_cores": os.cpu_count()}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 6),
+            "us_per_step": round(ms_per_step * 1e3, 3),
+            "pct_of_measured_hbm_peak": round(100 * per_gpu / peak, 2),
+            "pct_of_nominal_8tbs": round(100 * per_gpu / NOMINAL_HBM_GBS, 2),
+            "tokens_of_kv_per_s": round(total_keys * world / (ms_per_step * 1e-3), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
+            "config": {"workload": args.workload, "B": B, "H": H, "D": D, "N": N,
+                       "ragged": w.ragged is not None, "alibi": w.alibi,
+                       "n_split": n_split if n_split else "auto", "parts": parts,
+                       "bytes_per_step": int(bytes_step),
+                       "l2": "no flush: K+V per step %.2f GB > 126 MB L2" % (bytes_step / 1e9),
+                       "parallelism": "replicas x%d" % world},
+            "gpu_launches": args.steps, "clocks": clocks, "roofline": roofline,
+            "e2e": e2e, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# -------------------------------------------------------- reference arm
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w, "cpu")
+    # each step is a bounded sample so the whole run stays within ~2 minutes
+    per_step_budget = max(0.002, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_rate(inp, w, budget_s=per_step_budget)
+    t0 = time.perf_counter()
+    rates = []
+    desc, used = "", 1
+    for _ in range(args.steps):
+        r, used, desc, _ = oracle_rate(inp, w, budget_s=per_step_budget)
+        rates.append(r)
+    dt = time.perf_counter() - t0
+    value = sum(rates) / len(rates)
+    line = {
+        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * dt / args.steps, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.workload, "B": w.B, "H": w.H, "D": w.D, "N": w.N},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": used,
+                         "kind": "oracle", "sample": "per step: " + desc},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--n-split", type=int, default=None)
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

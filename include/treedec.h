@@ -1,0 +1,214 @@
+/*
+ * treedec.h -- C ABI of libtreedec: exact single-query (decode-step) softmax
+ * attention over a long KV sequence on one NVIDIA B200 (sm_100a).
+ *
+ * The computation is the decode scheme of the "Tree Attention Decoding" gist
+ * (tree_attn_decode.py, function tree_attn_decode, "Algorithm 3 proposed in
+ * Tree Attention"): the key/value sequence is cut into parts, each part yields
+ * a numerator num = sum_j e^(s_j - m) v_j, its local max m and denominator
+ * l = sum_j e^(s_j - m), and the parts are merged by rescaling with
+ * e^(m - max m) and summing (the gist's all-reduce MAX and two all-reduce
+ * SUMs; the softmax decomposition and fusion formulas of "Flash Aandacht",
+ * section "De Wiskunde Achter Flash Aandacht").  Here the parts are CTAs of
+ * one GPU and the merge runs on the GPU.  The result equals plain attention
+ * (the gist's regular_decode):
+ *
+ *   s_j  = (q . k_j) * D^-1/2 + slope_h * (j - n + 1)
+ *   out  = sum_j softmax(s)_j v_j        lse = ln sum_j e^(s_j)
+ *
+ * where the optional ALiBi term is the broadcast bias row arange(1-n, 1)
+ * times the head slope ("ALiBi with causal=True unexpected bias?",
+ * llm-foundry issue #186), computed in registers: no bias tensor is read.
+ *
+ * Conventions shared by every entry point
+ *   - Layout (row-major, contiguous): q [B,H,1,D], k and v [B,H,N,D],
+ *     out [B,H,1,D] fp32, lse [B,H,1] fp32.  Element type of q, k, v: dtype.
+ *   - Pointers named "device" must be CUDA device (or managed) memory on the
+ *     current device; the caller owns all of them.  q, k, v must be 16-byte
+ *     aligned; out, lse, slopes, seqlens 4-byte aligned.
+ *   - D must be 64, 128, 256 or 512.
+ *   - All work is enqueued on `stream`; no call synchronises the device
+ *     except td_check_device_error, td_release_workspace and td_decode_host
+ *     (which only waits on its own stream when asked to).
+ *   - Errors are returned as td_status; arguments are validated on the host
+ *     before anything is launched, and a rejected call launches nothing.
+ *   - The library-owned workspace is per device and grows on demand (a
+ *     cudaMalloc on growth: make the first call of a given size outside
+ *     stream capture).  Calls that share it must be ordered on one stream;
+ *     for concurrent streams give each its own workspace (td_decode_ws).
+ */
+#ifndef TREEDEC_H
+#define TREEDEC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TD_API __attribute__((visibility("default")))
+#else
+#define TD_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* The CUDA stream type (identical to cudaStream_t / CUstream). */
+struct CUstream_st;
+typedef struct CUstream_st *td_stream;
+
+typedef enum { TD_F32 = 0, TD_BF16 = 1, TD_F16 = 2 } td_dtype;
+
+typedef enum {
+    TD_OK = 0,
+    TD_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, overflow   */
+    TD_ERR_UNSUPPORTED = 2, /* D or dtype outside the compiled set           */
+    TD_ERR_CUDA = 3,        /* a CUDA runtime call failed: td_last_cuda_error */
+    TD_ERR_NO_MEMORY = 4,   /* workspace allocation failed                   */
+    TD_ERR_DEVICE = 5,      /* a kernel reported an error word (see below)    */
+    TD_ERR_WORKSPACE = 6    /* caller workspace too small                     */
+} td_status;
+
+/* Device error word bits reported through td_check_device_error. */
+#define TD_DEVERR_WAIT_TIMEOUT 0x1 /* a bounded pipeline wait ran out        */
+#define TD_DEVERR_BAD_SEQLEN 0x2   /* a seqlens[b] outside [0, Nmax], clamped */
+
+/*
+ * td_decode -- decode attention for every (b,h): q[b,h] against the N keys of
+ * k[b,h] and values of v[b,h]  (gist: tree_attn_decode / regular_decode).
+ *   q, k, v   device, dtype, layouts above.
+ *   out       device fp32 [B,H,1,D]; lse device fp32 [B,H,1] or NULL.
+ *   N >= 1    keys per sequence.
+ *   n_split   0: the library's split heuristic (td_auto_split) over the whole
+ *             flattened key space; > 0: each (b,h) is cut into
+ *             min(n_split, N) parts of balanced length (the gist's one chunk
+ *             per rank).  The result is the same to rounding either way.
+ *   alibi_slopes  device fp32 [H] (per-head slope) or NULL for no bias.
+ * Uses the library-owned per-device workspace.
+ */
+TD_API td_status td_decode(const void *q, const void *k, const void *v, float *out, float *lse,
+                    int B, int H, int64_t N, int D, int n_split,
+                    const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
+/*
+ * td_decode_varlen -- as td_decode for a batch of sequences of different
+ * lengths stored padded: k, v [B,H,Nmax,D]; sequence b attends to its first
+ * seqlens[b] keys and the ALiBi term uses n = seqlens[b].
+ *   seqlens       device int32 [B], 0 <= seqlens[b] <= Nmax (a value outside
+ *                 is clamped and flagged with TD_DEVERR_BAD_SEQLEN).  A length
+ *                 of 0 gives out = 0 and lse = -inf.
+ *   seqlens_host  optional host copy of the same lengths (or NULL); when given
+ *                 the heuristic sizes the split from the true key count.
+ *   n_split       0: heuristic; > 0: B*H*n_split parts over the flattened
+ *                 (b, h, key) space of attended keys.
+ * Keys at positions >= seqlens[b] are never read.
+ */
+TD_API td_status td_decode_varlen(const void *q, const void *k, const void *v, float *out,
+                           float *lse, int B, int H, int64_t Nmax, int D,
+                           const int32_t *seqlens, const int32_t *seqlens_host, int n_split,
+                           const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
+/*
+ * td_decode_ws -- the general form with a caller-owned workspace and an
+ * explicit part count.
+ *   seqlens / seqlens_host  as td_decode_varlen, or both NULL (every sequence
+ *                 has N keys).
+ *   parts         total number of parts over the flattened (b, h, key) space
+ *                 (one CTA each): 0 = heuristic.  Part c covers the flattened
+ *                 keys [floor(c*T/parts), floor((c+1)*T/parts)) where T is the
+ *                 number of attended keys; parts = B*H*n gives exactly n
+ *                 balanced parts per (b,h) when all lengths are equal.
+ *   workspace     device, at least td_workspace_bytes(B, H, D, parts_used)
+ *                 bytes (parts_used = the heuristic's value when parts = 0:
+ *                 ask td_plan_parts), zero-filled before its first use; the
+ *                 kernels leave it ready for the next call.  Calls sharing one
+ *                 workspace must be ordered on one stream.
+ */
+TD_API td_status td_decode_ws(const void *q, const void *k, const void *v, float *out, float *lse,
+                       int B, int H, int64_t N, int D, const int32_t *seqlens,
+                       const int32_t *seqlens_host, int64_t parts,
+                       const float *alibi_slopes, td_dtype dtype, void *workspace,
+                       size_t workspace_bytes, td_stream stream);
+
+/*
+ * td_combine -- merge caller-provided partials into the final output: the
+ * gist's global max, renormalisation and two sums (tree_attn_decode after
+ * "first get global max"), done per (b,h) as a log-depth tree on the GPU.
+ *   num   device fp32 [B,H,S,D]: sum_j e^(s_j - m_s) v_j of part s;
+ *   m     device fp32 [B,H,S]: the part's max score (natural-log units);
+ *   l     device fp32 [B,H,S]: sum_j e^(s_j - m_s).
+ *   An empty part is (num = 0, m = -inf, l = 0) and contributes nothing; if
+ *   every part of a (b,h) is empty its out is 0 and lse is -inf.
+ *   out   device fp32 [B,H,1,D]; lse device fp32 [B,H,1] or NULL.
+ *   1 <= D <= 1024, S >= 1.
+ */
+TD_API td_status td_combine(const float *num, const float *m, const float *l, float *out, float *lse,
+                     int B, int H, int S, int D, td_stream stream);
+
+/*
+ * td_auto_split -- the split heuristic: the number of parts (CTAs) for T =
+ * B*H*N attended keys on a GPU with num_sms SMs: enough to fill every SM with
+ * as many CTAs as fit at once, but no part smaller than 64 KiB of K+V and
+ * never more parts than keys.  Pure host arithmetic (no GPU needed).
+ * Returns -1 on invalid arguments.
+ */
+TD_API int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int num_sms);
+
+/*
+ * td_plan_parts -- the part count the decode entry points use on the current
+ * device.  total_keys < 0: equal lengths Nmax, td_decode's rule (n_split > 0
+ * gives B*H*min(n_split, Nmax) parts).  total_keys >= 0: ragged lengths
+ * summing to total_keys over all (b,h), td_decode_varlen's rule with
+ * seqlens_host given (n_split > 0 gives B*H*n_split parts).  Either way
+ * n_split = 0 means the heuristic, and the count is capped at the number of
+ * keys.  Returns -1 on invalid arguments or when no device is available.
+ */
+TD_API int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, int n_split,
+                      int64_t total_keys);
+
+/* Bytes of workspace td_decode_ws needs for `parts` parts. */
+TD_API size_t td_workspace_bytes(int B, int H, int D, int64_t parts);
+
+/*
+ * td_decode_host -- td_decode / td_decode_varlen with HOST buffers: copies
+ * q, k, v (and slopes, seqlens) to device staging owned by the library, runs
+ * the decode, and copies out and lse back, all on `stream`.  Host buffers
+ * should be pinned for the copies to be asynchronous.  seqlens (host int32
+ * [B]) may be NULL for equal lengths N.  If sync != 0 the call waits for the
+ * stream before returning (out/lse are then valid); otherwise the caller
+ * must synchronise `stream` before reading them.
+ */
+TD_API td_status td_decode_host(const void *q, const void *k, const void *v, float *out, float *lse,
+                         int B, int H, int64_t N, int D, const int32_t *seqlens,
+                         int n_split, const float *alibi_slopes, td_dtype dtype,
+                         td_stream stream, int sync);
+
+/*
+ * td_check_device_error -- wait for `stream`, then read and clear the device
+ * error word of the library-owned workspace on the current device (or of
+ * `workspace` when it is not NULL).  Returns TD_OK, or TD_ERR_DEVICE with the
+ * TD_DEVERR_* bits stored in *bits (if bits is not NULL).  After a device
+ * error the workspace's tickets are re-zeroed so the next call starts clean.
+ */
+TD_API td_status td_check_device_error(void *workspace, size_t workspace_bytes, int *bits,
+                                td_stream stream);
+
+/* Human-readable name of a status. */
+TD_API const char *td_status_string(td_status s);
+
+/* The last CUDA runtime error seen by this thread's calls (as an int
+ * cudaError_t), and clears it. */
+TD_API int td_last_cuda_error(void);
+
+/* Frees the library-owned workspaces and host-call staging on every device
+ * (waits for the device first). */
+TD_API void td_release_workspace(void);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+TD_API int td_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TREEDEC_H */

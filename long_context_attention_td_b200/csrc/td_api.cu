@@ -1,0 +1,429 @@
+// Host side of libtreedec: argument validation, the split heuristic, the
+// per-device workspace and staging buffers, and the extern "C" entry points
+// declared in treedec.h.  Nothing here computes attention: every step of the
+// decode runs in the kernels of td_partial.cu and td_combine.cu.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "td_internal.cuh"
+#include "treedec.h"
+
+namespace {
+
+thread_local int g_last_cuda = 0;
+std::mutex g_mu;
+
+struct DevState {
+    void* ws = nullptr;
+    size_t ws_bytes = 0;
+    void* stage = nullptr;  // device staging of td_decode_host
+    size_t stage_bytes = 0;
+    int num_sms = 0;
+};
+constexpr int kMaxDevices = 64;
+DevState g_dev[kMaxDevices];
+
+constexpr long long kLimit = 1LL << 62;
+
+td_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return TD_OK;
+    g_last_cuda = static_cast<int>(e);
+    return e == cudaErrorMemoryAllocation ? TD_ERR_NO_MEMORY : TD_ERR_CUDA;
+}
+
+bool dtype_ok(int t) { return t == TD_F32 || t == TD_BF16 || t == TD_F16; }
+int elt_size(int t) { return t == TD_F32 ? 4 : 2; }
+bool d_ok(int D) { return D == 64 || D == 128 || D == 256 || D == 512; }
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+// a * b <= kLimit for non-negative a, b
+bool mul_fits(long long a, long long b) { return a >= 0 && b >= 0 && (b == 0 || a <= kLimit / b); }
+
+size_t ticket_region(long long BH) { return align_up(static_cast<size_t>(BH) * 4, 256); }
+
+size_t ws_bytes_for(long long BH, int D, long long parts) {
+    return td::kErrRegion + ticket_region(BH) +
+           static_cast<size_t>(parts) * 2 * static_cast<size_t>(D + 2) * sizeof(float);
+}
+
+long long auto_parts(long long T, int D, int dtype, int num_sms) {
+    if (T <= 0) return 1;
+    const long long fill = static_cast<long long>(num_sms) * td::partial_ctas_per_sm(dtype, D);
+    const long long bytes_per_key = 2LL * D * elt_size(dtype);
+    long long by_size = T / (td::kMinPartBytes / bytes_per_key > 0
+                                 ? td::kMinPartBytes / bytes_per_key
+                                 : 1);
+    if (by_size < 1) by_size = 1;
+    long long P = fill < by_size ? fill : by_size;
+    if (P > T) P = T;
+    return P < 1 ? 1 : P;
+}
+
+td_status current_device(int* dev, int* num_sms) {
+    td_status st = cuda_status(cudaGetDevice(dev));
+    if (st != TD_OK) return st;
+    if (*dev < 0 || *dev >= kMaxDevices) return TD_ERR_UNSUPPORTED;
+    DevState& d = g_dev[*dev];
+    if (d.num_sms == 0) {
+        int n = 0;
+        st = cuda_status(cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, *dev));
+        if (st != TD_OK) return st;
+        d.num_sms = n;
+    }
+    *num_sms = d.num_sms;
+    return TD_OK;
+}
+
+// Grow the library-owned workspace of `dev` to at least `need` bytes.  A new
+// buffer is zero-filled on `stream` (the tickets must start at zero).
+td_status library_ws(int dev, size_t need, cudaStream_t stream, void** ws, size_t* bytes) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DevState& d = g_dev[dev];
+    if (d.ws_bytes < need) {
+        size_t nb = need < (size_t(1) << 20) ? (size_t(1) << 20) : need;
+        if (nb < 2 * d.ws_bytes) nb = 2 * d.ws_bytes;
+        if (d.ws) {
+            // cudaFree waits for outstanding work on the device first
+            cudaFree(d.ws);
+            d.ws = nullptr;
+            d.ws_bytes = 0;
+        }
+        void* p = nullptr;
+        td_status st = cuda_status(cudaMalloc(&p, nb));
+        if (st != TD_OK) return st;
+        st = cuda_status(cudaMemsetAsync(p, 0, nb, stream));
+        if (st != TD_OK) {
+            cudaFree(p);
+            return st;
+        }
+        d.ws = p;
+        d.ws_bytes = nb;
+    }
+    *ws = d.ws;
+    *bytes = d.ws_bytes;
+    return TD_OK;
+}
+
+struct Req {
+    const void *q, *k, *v;
+    float *out, *lse;
+    int B, H;
+    long long N;
+    int D;
+    const int32_t* seqlens;
+    const int32_t* seqlens_host;
+    long long parts;  // 0 = heuristic
+    const float* slopes;
+    int dtype;
+    void* ws;  // null = library-owned
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+td_status validate(const Req& r) {
+    if (!r.q || !r.k || !r.v || !r.out) return TD_ERR_INVALID_ARG;
+    if (!dtype_ok(r.dtype)) return TD_ERR_UNSUPPORTED;
+    if (r.B < 1 || r.H < 1 || r.N < 1 || r.D < 1 || r.parts < 0) return TD_ERR_INVALID_ARG;
+    if (!d_ok(r.D)) return TD_ERR_UNSUPPORTED;
+    if (!aligned(r.q, 16) || !aligned(r.k, 16) || !aligned(r.v, 16)) return TD_ERR_INVALID_ARG;
+    if (!aligned(r.out, 4) || (r.lse && !aligned(r.lse, 4)) ||
+        (r.slopes && !aligned(r.slopes, 4)) || (r.seqlens && !aligned(r.seqlens, 4)))
+        return TD_ERR_INVALID_ARG;
+    if (r.seqlens_host && !r.seqlens) return TD_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(r.B) * r.H;
+    if (BH > 0x7fffffffLL) return TD_ERR_INVALID_ARG;
+    if (!mul_fits(BH, r.N) || !mul_fits(BH * r.N, static_cast<long long>(r.D) * 4))
+        return TD_ERR_INVALID_ARG;
+    if (r.seqlens_host)
+        for (int b = 0; b < r.B; ++b)
+            if (r.seqlens_host[b] < 0 || r.seqlens_host[b] > r.N) return TD_ERR_INVALID_ARG;
+    return TD_OK;
+}
+
+// Attended keys when known on the host, else -1.
+long long known_keys(const Req& r) {
+    if (!r.seqlens) return static_cast<long long>(r.B) * r.H * r.N;
+    if (!r.seqlens_host) return -1;
+    long long s = 0;
+    for (int b = 0; b < r.B; ++b) s += r.seqlens_host[b];
+    return s * r.H;
+}
+
+long long plan_parts(const Req& r, int num_sms) {
+    const long long bound = static_cast<long long>(r.B) * r.H * r.N;
+    const long long known = known_keys(r);
+    const long long T = known >= 0 ? known : bound;
+    long long P = r.parts > 0 ? r.parts : auto_parts(T, r.D, r.dtype, num_sms);
+    const long long cap = T > 0 ? T : 1;
+    if (P > cap) P = cap;
+    if (P > 0x7fffffffLL) P = 0x7fffffffLL;
+    return P < 1 ? 1 : P;
+}
+
+td_status decode_impl(const Req& r) {
+    td_status st = validate(r);
+    if (st != TD_OK) return st;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TD_OK) return st;
+    const long long P = plan_parts(r, sms);
+    const long long BH = static_cast<long long>(r.B) * r.H;
+    if (!mul_fits(P + 1, BH * r.N)) return TD_ERR_INVALID_ARG;
+    const size_t need = ws_bytes_for(BH, r.D, P);
+    void* ws = r.ws;
+    size_t wsb = r.ws_bytes;
+    if (ws) {
+        if (!aligned(ws, 256)) return TD_ERR_INVALID_ARG;
+        if (wsb < need) return TD_ERR_WORKSPACE;
+    } else {
+        st = library_ws(dev, need, r.stream, &ws, &wsb);
+        if (st != TD_OK) return st;
+    }
+    char* base = static_cast<char*>(ws);
+    td::PartialParams p;
+    p.q = r.q;
+    p.k = r.k;
+    p.v = r.v;
+    p.out = r.out;
+    p.lse = r.lse;
+    p.slopes = r.slopes;
+    p.seqlens = r.seqlens;
+    p.B = r.B;
+    p.H = r.H;
+    p.N = r.N;
+    p.T = r.seqlens ? -1 : BH * r.N;
+    p.P = P;
+    p.qscale2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(r.D)));
+    p.err = reinterpret_cast<int*>(base);
+    p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
+    p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BH));
+    return cuda_status(td::launch_partial(r.dtype, r.D, p, r.stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+td_status td_decode(const void* q, const void* k, const void* v, float* out, float* lse, int B,
+                    int H, int64_t N, int D, int n_split, const float* alibi_slopes,
+                    td_dtype dtype, td_stream stream) {
+    if (n_split < 0) return TD_ERR_INVALID_ARG;
+    long long parts = 0;
+    if (n_split > 0) {
+        const long long per = n_split < N ? n_split : N;
+        parts = static_cast<long long>(B) * H * (per > 0 ? per : 1);
+    }
+    Req r{q, k, v, out, lse, B, H, N, D, nullptr, nullptr, parts, alibi_slopes,
+          static_cast<int>(dtype), nullptr, 0, reinterpret_cast<cudaStream_t>(stream)};
+    return decode_impl(r);
+}
+
+td_status td_decode_varlen(const void* q, const void* k, const void* v, float* out, float* lse,
+                           int B, int H, int64_t Nmax, int D, const int32_t* seqlens,
+                           const int32_t* seqlens_host, int n_split, const float* alibi_slopes,
+                           td_dtype dtype, td_stream stream) {
+    if (n_split < 0 || !seqlens) return TD_ERR_INVALID_ARG;
+    const long long parts = n_split > 0 ? static_cast<long long>(B) * H * n_split : 0;
+    Req r{q, k, v, out, lse, B, H, Nmax, D, seqlens, seqlens_host, parts, alibi_slopes,
+          static_cast<int>(dtype), nullptr, 0, reinterpret_cast<cudaStream_t>(stream)};
+    return decode_impl(r);
+}
+
+td_status td_decode_ws(const void* q, const void* k, const void* v, float* out, float* lse, int B,
+                       int H, int64_t N, int D, const int32_t* seqlens,
+                       const int32_t* seqlens_host, int64_t parts, const float* alibi_slopes,
+                       td_dtype dtype, void* workspace, size_t workspace_bytes,
+                       td_stream stream) {
+    if (!workspace || parts < 0) return TD_ERR_INVALID_ARG;
+    Req r{q, k, v, out, lse, B, H, N, D, seqlens, seqlens_host, parts, alibi_slopes,
+          static_cast<int>(dtype), workspace, workspace_bytes,
+          reinterpret_cast<cudaStream_t>(stream)};
+    return decode_impl(r);
+}
+
+td_status td_combine(const float* num, const float* m, const float* l, float* out, float* lse,
+                     int B, int H, int S, int D, td_stream stream) {
+    if (!num || !m || !l || !out) return TD_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || S < 1 || D < 1 || D > 1024) return TD_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(B) * H;
+    if (rows > 0x7fffffffLL || !mul_fits(rows * S, static_cast<long long>(D) * 4))
+        return TD_ERR_INVALID_ARG;
+    if (!aligned(num, 4) || !aligned(m, 4) || !aligned(l, 4) || !aligned(out, 4) ||
+        (lse && !aligned(lse, 4)))
+        return TD_ERR_INVALID_ARG;
+    return cuda_status(
+        td::launch_combine(num, m, l, out, lse, rows, S, D, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int num_sms) {
+    if (B < 1 || H < 1 || N < 1 || num_sms < 1 || !dtype_ok(dtype) || !d_ok(D)) return -1;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!mul_fits(BH, N)) return -1;
+    return auto_parts(BH * N, D, dtype, num_sms);
+}
+
+int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, int n_split,
+                      int64_t total_keys) {
+    if (B < 1 || H < 1 || Nmax < 1 || n_split < 0 || !dtype_ok(dtype) || !d_ok(D)) return -1;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!mul_fits(BH, Nmax)) return -1;
+    int dev = 0, sms = 0;
+    if (current_device(&dev, &sms) != TD_OK) return -1;
+    const long long bound = BH * Nmax;
+    long long T = total_keys >= 0 ? total_keys : bound;
+    if (T > bound) return -1;
+    long long parts = 0;
+    if (n_split > 0) {
+        const long long per = n_split < Nmax ? n_split : Nmax;
+        parts = total_keys < 0 ? BH * per : BH * n_split;
+    }
+    long long P = parts > 0 ? parts : auto_parts(T, D, dtype, sms);
+    const long long cap = T > 0 ? T : 1;
+    if (P > cap) P = cap;
+    return P < 1 ? 1 : P;
+}
+
+size_t td_workspace_bytes(int B, int H, int D, int64_t parts) {
+    if (B < 1 || H < 1 || D < 1 || parts < 1) return 0;
+    return ws_bytes_for(static_cast<long long>(B) * H, D, parts);
+}
+
+td_status td_decode_host(const void* q, const void* k, const void* v, float* out, float* lse,
+                         int B, int H, int64_t N, int D, const int32_t* seqlens, int n_split,
+                         const float* alibi_slopes, td_dtype dtype, td_stream stream, int sync) {
+    if (!q || !k || !v || !out || n_split < 0) return TD_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return TD_ERR_UNSUPPORTED;
+    if (B < 1 || H < 1 || N < 1) return TD_ERR_INVALID_ARG;
+    if (!d_ok(D)) return TD_ERR_UNSUPPORTED;
+    const long long BH = static_cast<long long>(B) * H;
+    if (!mul_fits(BH, N) || !mul_fits(BH * N, static_cast<long long>(D) * 4))
+        return TD_ERR_INVALID_ARG;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const size_t es = static_cast<size_t>(elt_size(dtype));
+    const size_t qb = static_cast<size_t>(BH) * D * es;
+    const size_t kvb = static_cast<size_t>(BH) * static_cast<size_t>(N) * D * es;
+    const size_t ob = static_cast<size_t>(BH) * D * sizeof(float);
+    const size_t lb = static_cast<size_t>(BH) * sizeof(float);
+    const size_t sb = alibi_slopes ? static_cast<size_t>(H) * sizeof(float) : 0;
+    const size_t nb = seqlens ? static_cast<size_t>(B) * sizeof(int32_t) : 0;
+    size_t off[7];
+    size_t total = 0;
+    const size_t sizes[7] = {qb, kvb, kvb, ob, lb, sb, nb};
+    for (int i = 0; i < 7; ++i) {
+        off[i] = total;
+        total += align_up(sizes[i] ? sizes[i] : 1, 256);
+    }
+    int dev = 0, sms = 0;
+    td_status st = current_device(&dev, &sms);
+    if (st != TD_OK) return st;
+    char* base = nullptr;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        DevState& d = g_dev[dev];
+        if (d.stage_bytes < total) {
+            if (d.stage) cudaFree(d.stage);
+            d.stage = nullptr;
+            d.stage_bytes = 0;
+            void* p = nullptr;
+            st = cuda_status(cudaMalloc(&p, total));
+            if (st != TD_OK) return st;
+            d.stage = p;
+            d.stage_bytes = total;
+        }
+        base = static_cast<char*>(d.stage);
+    }
+    const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
+    st = cuda_status(cudaMemcpyAsync(base + off[0], q, qb, h2d, s));
+    if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[1], k, kvb, h2d, s));
+    if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[2], v, kvb, h2d, s));
+    if (st == TD_OK && sb) st = cuda_status(cudaMemcpyAsync(base + off[5], alibi_slopes, sb, h2d, s));
+    if (st == TD_OK && nb) st = cuda_status(cudaMemcpyAsync(base + off[6], seqlens, nb, h2d, s));
+    if (st != TD_OK) return st;
+    float* dout = reinterpret_cast<float*>(base + off[3]);
+    float* dlse = reinterpret_cast<float*>(base + off[4]);
+    const float* dsl = sb ? reinterpret_cast<const float*>(base + off[5]) : nullptr;
+    const int32_t* dsq = nb ? reinterpret_cast<const int32_t*>(base + off[6]) : nullptr;
+    if (dsq)
+        st = td_decode_varlen(base + off[0], base + off[1], base + off[2], dout, dlse, B, H, N, D,
+                              dsq, seqlens, n_split, dsl, dtype, stream);
+    else
+        st = td_decode(base + off[0], base + off[1], base + off[2], dout, dlse, B, H, N, D,
+                       n_split, dsl, dtype, stream);
+    if (st != TD_OK) return st;
+    st = cuda_status(cudaMemcpyAsync(out, dout, ob, cudaMemcpyDeviceToHost, s));
+    if (st == TD_OK && lse) st = cuda_status(cudaMemcpyAsync(lse, dlse, lb, cudaMemcpyDeviceToHost, s));
+    if (st == TD_OK && sync) st = cuda_status(cudaStreamSynchronize(s));
+    return st;
+}
+
+td_status td_check_device_error(void* workspace, size_t workspace_bytes, int* bits,
+                                td_stream stream) {
+    if (bits) *bits = 0;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    td_status st = cuda_status(cudaStreamSynchronize(s));
+    if (st != TD_OK) return st;
+    void* ws = workspace;
+    size_t wsb = workspace_bytes;
+    if (!ws) {
+        int dev = 0, sms = 0;
+        st = current_device(&dev, &sms);
+        if (st != TD_OK) return st;
+        std::lock_guard<std::mutex> lk(g_mu);
+        ws = g_dev[dev].ws;
+        wsb = g_dev[dev].ws_bytes;
+    }
+    if (!ws) return TD_OK;
+    if (wsb < td::kErrRegion) return TD_ERR_INVALID_ARG;
+    int h = 0;
+    st = cuda_status(cudaMemcpy(&h, ws, sizeof(int), cudaMemcpyDeviceToHost));
+    if (st != TD_OK) return st;
+    if (h == 0) return TD_OK;
+    if (bits) *bits = h;
+    st = cuda_status(cudaMemset(ws, 0, wsb));
+    if (st != TD_OK) return st;
+    return TD_ERR_DEVICE;
+}
+
+const char* td_status_string(td_status s) {
+    switch (s) {
+        case TD_OK: return "ok";
+        case TD_ERR_INVALID_ARG: return "invalid argument";
+        case TD_ERR_UNSUPPORTED: return "unsupported head size or element type";
+        case TD_ERR_CUDA: return "CUDA runtime error";
+        case TD_ERR_NO_MEMORY: return "out of device memory";
+        case TD_ERR_DEVICE: return "kernel reported an error";
+        case TD_ERR_WORKSPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+int td_last_cuda_error(void) {
+    const int e = g_last_cuda;
+    g_last_cuda = 0;
+    return e;
+}
+
+void td_release_workspace(void) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return;
+    for (int d = 0; d < kMaxDevices; ++d) {
+        DevState& s = g_dev[d];
+        if (!s.ws && !s.stage) continue;
+        if (cudaSetDevice(d) != cudaSuccess) continue;
+        cudaDeviceSynchronize();
+        if (s.ws) cudaFree(s.ws);
+        if (s.stage) cudaFree(s.stage);
+        s.ws = s.stage = nullptr;
+        s.ws_bytes = s.stage_bytes = 0;
+    }
+    cudaSetDevice(cur);
+}
+
+int td_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,57 @@
+// Internal declarations shared by the kernels and the host entry points of
+// libtreedec.  Not part of the C ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace td {
+
+// Element types (same numbering as td_dtype).
+enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+
+// Consumer warps per CTA of the split-KV kernel, plus one producer warp.
+constexpr int kConsumerWarps = 8;
+constexpr int kConsumerThreads = 32 * kConsumerWarps;
+constexpr int kPartialThreads = kConsumerThreads + 32;
+// Pipeline depth of the split-KV kernel (stages of K+V tiles in shared memory).
+constexpr int kStages = 4;
+// Bytes of K+V rows one pipeline stage holds (the tile is sized to this).
+constexpr int kStageBytes = 32768;
+// Smallest part the heuristic creates (bytes of K+V).
+constexpr int64_t kMinPartBytes = 65536;
+
+// Workspace layout: [error word | pad to 256 B][tickets: B*H int32, padded to
+// 256 B][part records: parts * 2 * (D + 2) fp32].
+constexpr size_t kErrRegion = 256;
+
+struct PartialParams {
+    const void* q;
+    const void* k;
+    const void* v;
+    float* out;
+    float* lse;              // may be null
+    const float* slopes;     // may be null
+    const int32_t* seqlens;  // null: every sequence has N keys
+    int B, H;
+    int64_t N;               // keys per sequence, or the padded Nmax when ragged
+    int64_t T;               // total attended keys when known (uniform), else -1
+    int64_t P;               // parts == grid size
+    float qscale2;           // D^-1/2 * log2(e)
+    float* part;             // part records
+    int* tickets;            // [B*H]
+    int* err;                // error word
+};
+
+// Dynamic shared memory of the split-KV kernel for (dtype, D).
+size_t partial_smem_bytes(int dtype, int D);
+// CTAs of the split-KV kernel that fit on one SM (static estimate from shared
+// memory and threads; matches the kernel's launch bounds).
+int partial_ctas_per_sm(int dtype, int D);
+// Launch the split-KV kernel (grid = p.P) with its fused combine.
+cudaError_t launch_partial(int dtype, int D, const PartialParams& p, cudaStream_t s);
+// Launch the standalone tree combine over dense partials.
+cudaError_t launch_combine(const float* num, const float* m, const float* l, float* out,
+                           float* lse, int64_t rows, int S, int D, cudaStream_t s);
+
+}  // namespace td
