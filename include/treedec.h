@@ -121,7 +121,9 @@ TD_API td_status td_decode_varlen(const void *q, const void *k, const void *v, f
  *   workspace     device, at least td_workspace_bytes(B, H, D, parts_used)
  *                 bytes (parts_used = the heuristic's value when parts = 0:
  *                 ask td_plan_parts), zero-filled before its first use; the
- *                 kernels leave it ready for the next call.  Calls sharing one
+ *                 kernels leave it ready for the next call (a call with a
+ *                 larger B*H than the workspace has served re-zeroes its
+ *                 ticket region on `stream` first).  Calls sharing one
  *                 workspace must be ordered on one stream.
  */
 TD_API td_status td_decode_ws(const void *q, const void *k, const void *v, float *out, float *lse,

@@ -29,6 +29,43 @@ DevState g_dev[kMaxDevices];
 
 constexpr long long kLimit = 1LL << 62;
 
+// Per workspace (library- or caller-owned): how many leading tickets are
+// known to be zero.  The kernels return every ticket they use to zero, but the
+// part records start right after the B*H tickets, so a later call with a
+// larger B*H finds part-record bytes where its new tickets go; those calls
+// zero the ticket region on the stream first.
+struct KnownZero {
+    const void* ws;
+    long long tickets;
+};
+constexpr int kMaxKnown = 256;
+KnownZero g_known[kMaxKnown];
+int g_known_n = 0;
+
+KnownZero* known_entry(const void* ws) {
+    for (int i = 0; i < g_known_n; ++i)
+        if (g_known[i].ws == ws) return &g_known[i];
+    return nullptr;
+}
+
+void forget_workspace(const void* ws) {
+    for (int i = 0; i < g_known_n; ++i)
+        if (g_known[i].ws == ws) {
+            g_known[i] = g_known[--g_known_n];
+            return;
+        }
+}
+
+void remember_workspace(const void* ws, long long tickets) {
+    KnownZero* e = known_entry(ws);
+    if (!e) {
+        if (g_known_n == kMaxKnown) g_known_n = kMaxKnown - 1;  // drop one: it gets re-zeroed
+        e = &g_known[g_known_n++];
+        e->ws = ws;
+    }
+    e->tickets = tickets;
+}
+
 td_status cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return TD_OK;
     g_last_cuda = static_cast<int>(e);
@@ -89,6 +126,7 @@ td_status library_ws(int dev, size_t need, cudaStream_t stream, void** ws, size_
         if (d.ws) {
             // cudaFree waits for outstanding work on the device first
             cudaFree(d.ws);
+            forget_workspace(d.ws);
             d.ws = nullptr;
             d.ws_bytes = 0;
         }
@@ -102,6 +140,7 @@ td_status library_ws(int dev, size_t need, cudaStream_t stream, void** ws, size_
         }
         d.ws = p;
         d.ws_bytes = nb;
+        remember_workspace(p, static_cast<long long>((nb - td::kErrRegion) / 4));
     }
     *ws = d.ws;
     *bytes = d.ws_bytes;
@@ -184,6 +223,16 @@ td_status decode_impl(const Req& r) {
         if (st != TD_OK) return st;
     }
     char* base = static_cast<char*>(ws);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const KnownZero* e = known_entry(ws);
+        if (!e || e->tickets < BH) {
+            st = cuda_status(
+                cudaMemsetAsync(base + td::kErrRegion, 0, ticket_region(BH), r.stream));
+            if (st != TD_OK) return st;
+        }
+        remember_workspace(ws, BH);
+    }
     td::PartialParams p;
     p.q = r.q;
     p.k = r.k;
@@ -385,6 +434,10 @@ td_status td_check_device_error(void* workspace, size_t workspace_bytes, int* bi
     if (bits) *bits = h;
     st = cuda_status(cudaMemset(ws, 0, wsb));
     if (st != TD_OK) return st;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        remember_workspace(ws, static_cast<long long>((wsb - td::kErrRegion) / 4));
+    }
     return TD_ERR_DEVICE;
 }
 
@@ -416,7 +469,10 @@ void td_release_workspace(void) {
         if (!s.ws && !s.stage) continue;
         if (cudaSetDevice(d) != cudaSuccess) continue;
         cudaDeviceSynchronize();
-        if (s.ws) cudaFree(s.ws);
+        if (s.ws) {
+            cudaFree(s.ws);
+            forget_workspace(s.ws);
+        }
         if (s.stage) cudaFree(s.stage);
         s.ws = s.stage = nullptr;
         s.ws_bytes = s.stage_bytes = 0;

@@ -150,6 +150,28 @@ def test_repeated_calls_are_bitwise_identical_and_tickets_reset():
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
 
 
+def test_workspace_reuse_with_growing_and_shrinking_batch():
+    """One workspace (library-owned, then caller-owned) serving calls whose
+    B*H goes up and down: the ticket region must be zero whenever it grows
+    over memory earlier calls used for part records."""
+    shapes = [(1, 2, 5000), (64, 16, 40), (1, 3, 7000), (128, 16, 33), (2, 2, 900),
+              (128, 16, 33)]
+    cases = []
+    for i, (B, H, N) in enumerate(shapes):
+        w = Workload("reuse%d" % i, torch.bfloat16, B, H, 128, N, seed=60 + i)
+        inp = make_inputs(w, DEV)
+        cases.append((w, inp, oracle_all(inp)))
+    for w, inp, (ro, rl) in cases:
+        out, lse = run_td(inp)
+        compare(out, lse, ro, rl, np.arange(w.B * w.H), w.dtype)
+    ws = torch.zeros(4 << 20, dtype=torch.uint8, device=DEV)
+    for w, inp, (ro, rl) in cases + cases[::-1]:
+        for P in (37, 300):
+            out, lse = td.decode_ws(inp["q"], inp["k"], inp["v"], ws, parts=P)
+            td.check_device_error(ws)
+            compare(out, lse, ro, rl, np.arange(w.B * w.H), w.dtype)
+
+
 def test_caller_workspace_matches_library_workspace():
     w = Workload("ws", torch.bfloat16, 1, 4, 128, 9000, seed=31)
     inp = make_inputs(w, DEV)
