@@ -168,6 +168,39 @@ TD_API int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int
 TD_API int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, int n_split,
                       int64_t total_keys);
 
+/*
+ * td_decode_static -- td_decode that allocates nothing.  (The pages have no
+ * counterpart: this entry point exists for callers of the library, not for
+ * the method.)  Some callers cannot allocate device memory: serving engines
+ * that reserve nearly all HBM for their KV-cache pool up front (a cudaMalloc
+ * would fail or fragment the pool), host applications that own every device
+ * allocation of a plug-in, and latency-critical decode loops that cannot
+ * absorb the device-wide synchronisation of cudaMalloc/cudaFree.
+ *   Arguments, layouts, results and error returns are those of td_decode; the
+ *   caller still provides q, k, v, out and lse.  The workspace is a fixed
+ *   array of TD_STATIC_SCRATCH_BYTES inside the library's device image (every
+ *   GPU that loads the library holds it until the process exits); no
+ *   cudaMalloc, cudaFree or other allocating routine is called.
+ *   - A problem whose workspace (td_workspace_bytes for the part count
+ *     td_plan_parts gives) exceeds TD_STATIC_SCRATCH_BYTES is rejected with
+ *     TD_ERR_WORKSPACE before anything is launched (for example bf16, D=128
+ *     with the heuristic split fits for B*H up to about 200,000; very large
+ *     explicit n_split values may not).
+ *   - The first call on a device sets up that device (looks up the array's
+ *     address and zero-fills it, synchronously); make that first call before
+ *     any stream capture.
+ *   - Every call on a device shares the one array and it keeps the last call's
+ *     contents (tickets are left at zero by each call).  Calls that overlap on
+ *     the GPU -- on different streams, or from different threads without
+ *     ordering -- race on it and give wrong results: order them on one stream.
+ *   - Device error bits of these calls stay in the array and are not reported
+ *     by td_check_device_error.
+ */
+#define TD_STATIC_SCRATCH_BYTES (1u << 20)
+TD_API td_status td_decode_static(const void *q, const void *k, const void *v, float *out,
+                                  float *lse, int B, int H, int64_t N, int D, int n_split,
+                                  const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
 /* Bytes of workspace td_decode_ws needs for `parts` parts. */
 TD_API size_t td_workspace_bytes(int B, int H, int D, int64_t parts);
 
