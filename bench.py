@@ -239,6 +239,8 @@ def run_ours(args):
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
     w = w.with_(seed=w.seed + 1000 * rank)
+    if args.n_keys:
+        w = w.with_(N=args.n_keys)
     inp = make_inputs(w, dev)
     q, k, v = inp["q"], inp["k"], inp["v"]
     n_split = w.n_split if args.n_split is None else args.n_split
@@ -364,7 +366,8 @@ def run_ours(args):
             "tokens_of_kv_per_s": round(total_keys * world / (ms_per_step * 1e-3), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
-            "config": {"workload": args.workload, "B": B, "H": H, "D": D, "N": N,
+            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
+                       "B": B, "H": H, "D": D, "N": N,
                        "ragged": w.ragged is not None, "alibi": w.alibi,
                        "n_split": n_split if n_split else "auto", "parts": parts,
                        "bytes_per_step": int(bytes_step),
@@ -423,6 +426,8 @@ def main(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--n-split", type=int, default=None)
+    ap.add_argument("--n-keys", type=int, default=0,
+                    help="override keys per sequence (smaller profiling captures)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")

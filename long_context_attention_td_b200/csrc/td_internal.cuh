@@ -10,14 +10,31 @@ namespace td {
 // Element types (same numbering as td_dtype).
 enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 
+// Shape of the split-KV kernel's pipeline (compile-time; the defaults are the
+// tuned values, the macros exist for tuning sweeps).
+#ifndef TD_CONSUMER_WARPS
+#define TD_CONSUMER_WARPS 8
+#endif
+#ifndef TD_STAGES
+#define TD_STAGES 4
+#endif
+#ifndef TD_STAGE_BYTES
+#define TD_STAGE_BYTES 32768
+#endif
+#ifndef TD_CTAS_PER_SM
+#define TD_CTAS_PER_SM 1
+#endif
+
 // Consumer warps per CTA of the split-KV kernel, plus one producer warp.
-constexpr int kConsumerWarps = 8;
+constexpr int kConsumerWarps = TD_CONSUMER_WARPS;
 constexpr int kConsumerThreads = 32 * kConsumerWarps;
 constexpr int kPartialThreads = kConsumerThreads + 32;
 // Pipeline depth of the split-KV kernel (stages of K+V tiles in shared memory).
-constexpr int kStages = 4;
+constexpr int kStages = TD_STAGES;
 // Bytes of K+V rows one pipeline stage holds (the tile is sized to this).
-constexpr int kStageBytes = 32768;
+constexpr int kStageBytes = TD_STAGE_BYTES;
+// CTAs of the split-KV kernel meant to share one SM (launch bounds).
+constexpr int kCtasPerSm = TD_CTAS_PER_SM;
 // Smallest part the heuristic creates (bytes of K+V).
 constexpr int64_t kMinPartBytes = 65536;
 

@@ -42,7 +42,7 @@ struct Cfg {
     static constexpr int kGPW = 32 / kG;                        // row groups per warp
     static constexpr int kNG = kConsumerWarps * kGPW;           // row groups per CTA
     static constexpr int kRPGraw = (kStageBytes / 2) / (kNG * kRowBytes);
-    static constexpr int kRPG = kRPGraw < 1 ? 1 : (kRPGraw > 4 ? 4 : kRPGraw);
+    static constexpr int kRPG = kRPGraw < 1 ? 1 : (kRPGraw > 8 ? 8 : kRPGraw);
     static constexpr int kTile = kRPG * kNG;                    // key rows per stage
     static constexpr int kTileBytes = kTile * kRowBytes;        // K (or V) bytes per stage
     static constexpr int kStage = 2 * kTileBytes;
@@ -143,7 +143,7 @@ struct SlotAcc {
 constexpr int kBarConsumers = 1;
 
 template <typename E, int D>
-__global__ void __launch_bounds__(kPartialThreads, 1) td_partial_kernel(const PartialParams p) {
+__global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel(const PartialParams p) {
     using C = Cfg<E, D>;
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -547,6 +547,7 @@ int partial_ctas_per_sm(int dtype, int D) {
     int by_smem = static_cast<int>((228u * 1024u) / per_cta);
     const int by_threads = 2048 / kPartialThreads;
     int n = by_smem < by_threads ? by_smem : by_threads;
+    if (n > kCtasPerSm) n = kCtasPerSm;
     return n < 1 ? 1 : n;
 }
 
