@@ -1,0 +1,120 @@
+"""Multi-process paths on CPU ranks (gloo, world size 2 and 3).
+
+1. The gist's own scheme ("Tree Attention Decoding", tree_attn_decode): every
+   rank owns one chunk of the keys (k.chunk(world_size)), computes its
+   (num, local_max, den) with the oracle, then all-reduce MAX, renormalise and
+   two all-reduce SUMs -- the result must equal the plain definition.
+2. bench.py's rank aggregation: max of the timed region over ranks, sum of the
+   work, and one JSON line from rank 0 only.
+"""
+import math
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _init(rank, world, port):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+
+
+def _gist_scheme(rank, world, port, n, D, slope, q, k, v, result):
+    import oracle
+    _init(rank, world, port)
+    try:
+        starts = oracle.chunk_bounds(n, world, "torch_chunk")
+        j0, j1 = starts[rank], starts[rank + 1]
+        num, m, den = oracle.chunk_partial(q, k, v, j0, j1, slope=slope)
+        num = torch.from_numpy(num)
+        gmax = torch.tensor([m], dtype=torch.float64)
+        dist.all_reduce(gmax, op=dist.ReduceOp.MAX)
+        r = math.exp(m - float(gmax)) if m != -math.inf else 0.0
+        den_t = torch.tensor([den * r], dtype=torch.float64)
+        num_t = num * r
+        dist.all_reduce(den_t)
+        dist.all_reduce(num_t)
+        out = (num_t / den_t).numpy()
+        if rank == 0:
+            result.put((out.tolist(), float(gmax) + math.log(float(den_t))))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n", [(2, 31), (3, 31), (2, 1)])
+def test_gist_allreduce_scheme_on_cpu_ranks(world, n):
+    import oracle
+    D = 64
+    g = torch.Generator().manual_seed(world * 100 + n)
+    q = sum(torch.randn(D, generator=g) for _ in range(world))
+    k = sum(torch.randn(n, D, generator=g) for _ in range(world))
+    v = sum(torch.randn(n, D, generator=g) for _ in range(world))
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gist_scheme, args=(r, world, port, n, D, 0.25, q, k, v, result))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    out, lse = result.get(timeout=120)
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    ref, ref_l = oracle.attend_one(q, k, v, slope=0.25)
+    np.testing.assert_allclose(np.array(out), ref, rtol=0, atol=1e-12)
+    assert abs(lse - ref_l) < 1e-12
+
+
+def _bench_aggregate(rank, world, port, result):
+    import bench
+    _init(rank, world, port)
+    try:
+        ms = [3.0, 5.0, 4.0][rank]
+        mx = bench.reduce_max(ms, "cpu")
+        tot = bench.reduce_sum(100.0 * (rank + 1), "cpu")
+        bench.barrier()
+        result.put((rank, mx, tot))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_bench_takes_the_max_time_and_sums_work_over_ranks(world):
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_aggregate, args=(r, world, port, result))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted(result.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    expect_max = max([3.0, 5.0, 4.0][:world])
+    expect_sum = sum(100.0 * (r + 1) for r in range(world))
+    for rank, mx, tot in got:
+        assert mx == expect_max and tot == expect_sum
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    import bench
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
+    assert capsys.readouterr().out == ""
