@@ -298,27 +298,25 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         const bool whole = (j0 == 0 && j1 == w.len);
         const long long bh = static_cast<long long>(w.b) * p.H + w.h;
 
-        float qf[C::kNV][C::kVec];
+        // q stays in its input element type; the scale goes on the finished sum
+        uint4 qv[C::kNV];
         {
             const E* qrow = static_cast<const E*>(p.q) + bh * D;
 #pragma unroll
-            for (int u = 0; u < C::kNV; ++u) {
-                const uint4 r =
-                    __ldg(reinterpret_cast<const uint4*>(qrow + (u * C::kG + lig) * C::kVec));
-                Elem<E>::to_f32(r, qf[u]);
-#pragma unroll
-                for (int x = 0; x < C::kVec; ++x) qf[u][x] *= p.qscale2;
-            }
+            for (int u = 0; u < C::kNV; ++u)
+                qv[u] = __ldg(reinterpret_cast<const uint4*>(qrow + (u * C::kG + lig) * C::kVec));
         }
+        const float qscale2 = p.qscale2;
         const bool has_bias = p.slopes != nullptr;
         const float slope2 = has_bias ? __ldg(p.slopes + w.h) * kLog2e : 0.f;
 
+        constexpr int kPairs = C::kVec / 2;  // fp32 pairs per 16-byte vector
         float m = kNegInf, l = 0.f;
-        float acc[C::kNV][C::kVec];
+        uint64_t acc[C::kNV][kPairs];
 #pragma unroll
         for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-            for (int x = 0; x < C::kVec; ++x) acc[u][x] = 0.f;
+            for (int x = 0; x < kPairs; ++x) acc[u][x] = 0ull;
 
         for (long long t0 = j0; t0 < j1; t0 += C::kTile) {
             const long long left = j1 - t0;
@@ -336,13 +334,9 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 float a = 0.f;
                 if (row < rows) {
 #pragma unroll
-                    for (int u = 0; u < C::kNV; ++u) {
-                        const uint4 r = lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16);
-                        float kf[C::kVec];
-                        Elem<E>::to_f32(r, kf);
-#pragma unroll
-                        for (int x = 0; x < C::kVec; ++x) a = fmaf(qf[u][x], kf[x], a);
-                    }
+                    for (int u = 0; u < C::kNV; ++u)
+                        a = RowMath<E>::dot(
+                            qv[u], lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16), a);
                 }
                 s[i] = a;
             }
@@ -356,8 +350,9 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             for (int i = 0; i < C::kRPG; ++i) {
                 const int row = gi + i * C::kNG;
                 if (row < rows) {
-                    if (has_bias)
-                        s[i] = fmaf(slope2, static_cast<float>(t0 + row - w.len + 1), s[i]);
+                    s[i] = has_bias
+                               ? fmaf(s[i], qscale2, slope2 * static_cast<float>(t0 + row - w.len + 1))
+                               : s[i] * qscale2;
                     tmax = fmaxf(tmax, s[i]);
                 } else {
                     s[i] = kNegInf;
@@ -367,25 +362,22 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 const float mn = fmaxf(m, tmax);
                 const float alpha = rescale(m, mn);
                 l *= alpha;
+                const uint64_t aa = pack2(alpha, alpha);
 #pragma unroll
                 for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-                    for (int x = 0; x < C::kVec; ++x) acc[u][x] *= alpha;
+                    for (int x = 0; x < kPairs; ++x) acc[u][x] = mul2(acc[u][x], aa);
 #pragma unroll
                 for (int i = 0; i < C::kRPG; ++i) {
                     const int row = gi + i * C::kNG;
                     if (row < rows) {
                         const float pr = ex2(s[i] - mn);
                         l += pr;
+                        const uint64_t pp = pack2(pr, pr);
 #pragma unroll
-                        for (int u = 0; u < C::kNV; ++u) {
-                            const uint4 r =
-                                lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16);
-                            float vf[C::kVec];
-                            Elem<E>::to_f32(r, vf);
-#pragma unroll
-                            for (int x = 0; x < C::kVec; ++x) acc[u][x] = fmaf(pr, vf[x], acc[u][x]);
-                        }
+                        for (int u = 0; u < C::kNV; ++u)
+                            RowMath<E>::pv(acc[u], pp,
+                                           lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16));
                     }
                 }
                 m = mn;
@@ -399,6 +391,15 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         }
 
         // ---- end of piece: merge the row groups of the warp (xor butterfly)
+        float accf[C::kNV][C::kVec];
+#pragma unroll
+        for (int u = 0; u < C::kNV; ++u)
+#pragma unroll
+            for (int x = 0; x < kPairs; ++x) {
+                const float2 f = unpack2(acc[u][x]);
+                accf[u][2 * x] = f.x;
+                accf[u][2 * x + 1] = f.y;
+            }
 #pragma unroll
         for (int o = C::kG; o < 32; o <<= 1) {
             const float mo = __shfl_xor_sync(0xffffffffu, m, o);
@@ -410,8 +411,8 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
                 for (int x = 0; x < C::kVec; ++x) {
-                    const float ao = __shfl_xor_sync(0xffffffffu, acc[u][x], o);
-                    acc[u][x] = acc[u][x] * a + ao * b;
+                    const float ao = __shfl_xor_sync(0xffffffffu, accf[u][x], o);
+                    accf[u][x] = accf[u][x] * a + ao * b;
                 }
             m = M;
         }
@@ -420,7 +421,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
 #pragma unroll
             for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-                for (int x = 0; x < C::kVec; ++x) rw[(u * C::kG + lig) * C::kVec + x] = acc[u][x];
+                for (int x = 0; x < C::kVec; ++x) rw[(u * C::kG + lig) * C::kVec + x] = accf[u][x];
             if (lane == 0) {
                 rw[D] = m;
                 rw[D + 1] = l;
