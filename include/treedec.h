@@ -142,7 +142,7 @@ TD_API td_status td_decode_ws(const void *q, const void *k, const void *v, float
  *   An empty part is (num = 0, m = -inf, l = 0) and contributes nothing; if
  *   every part of a (b,h) is empty its out is 0 and lse is -inf.
  *   out   device fp32 [B,H,1,D]; lse device fp32 [B,H,1] or NULL.
- *   1 <= D <= 1024, S >= 1.
+ *   1 <= D <= 512, S >= 1.
  */
 TD_API td_status td_combine(const float *num, const float *m, const float *l, float *out, float *lse,
                      int B, int H, int S, int D, td_stream stream);
@@ -183,9 +183,9 @@ TD_API int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, 
  *   cudaMalloc, cudaFree or other allocating routine is called.
  *   - A problem whose workspace (td_workspace_bytes for the part count
  *     td_plan_parts gives) exceeds TD_STATIC_SCRATCH_BYTES is rejected with
- *     TD_ERR_WORKSPACE before anything is launched (for example bf16, D=128
- *     with the heuristic split fits for B*H up to about 200,000; very large
- *     explicit n_split values may not).
+ *     TD_ERR_WORKSPACE before anything is launched (with the heuristic split
+ *     on a B200 every D fits for B*H up to about 60,000, and D=128 up to about
+ *     400,000; very large explicit n_split values may not).
  *   - The first call on a device sets up that device (looks up the array's
  *     address and zero-fills it, synchronously); make that first call before
  *     any stream capture.
@@ -196,7 +196,7 @@ TD_API int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, 
  *   - Device error bits of these calls stay in the array and are not reported
  *     by td_check_device_error.
  */
-#define TD_STATIC_SCRATCH_BYTES (1u << 20)
+#define TD_STATIC_SCRATCH_BYTES (2u << 20)
 TD_API td_status td_decode_static(const void *q, const void *k, const void *v, float *out,
                                   float *lse, int B, int H, int64_t N, int D, int n_split,
                                   const float *alibi_slopes, td_dtype dtype, td_stream stream);

@@ -297,7 +297,7 @@ td_status td_decode_ws(const void* q, const void* k, const void* v, float* out, 
 td_status td_combine(const float* num, const float* m, const float* l, float* out, float* lse,
                      int B, int H, int S, int D, td_stream stream) {
     if (!num || !m || !l || !out) return TD_ERR_INVALID_ARG;
-    if (B < 1 || H < 1 || S < 1 || D < 1 || D > 1024) return TD_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || S < 1 || D < 1 || D > 512) return TD_ERR_INVALID_ARG;
     const long long rows = static_cast<long long>(B) * H;
     if (rows > 0x7fffffffLL || !mul_fits(rows * S, static_cast<long long>(D) * 4))
         return TD_ERR_INVALID_ARG;

@@ -13,6 +13,7 @@ namespace {
 using namespace dev;
 
 constexpr int kCombineThreads = 256;
+constexpr int kCombineScratch = 2048;  // weights of up to 2048 parts per chunk
 
 // Dense caller layout: num [rows, S, D], m and l [rows, S], m in natural-log
 // units (converted to the log2 units of tree_merge).
@@ -32,11 +33,11 @@ struct DenseAcc {
 __global__ void __launch_bounds__(kCombineThreads) td_tree_combine_kernel(
     const float* __restrict__ num, const float* __restrict__ m, const float* __restrict__ l,
     float* __restrict__ out, float* __restrict__ lse, int S, int D) {
-    __shared__ float scratch[kCombineThreads];
+    __shared__ float scratch[kCombineScratch];
     const long long row = blockIdx.x;
     const DenseAcc acc{num, m, l, row, S, D};
-    tree_merge(acc, S, D, static_cast<int>(threadIdx.x), kCombineThreads, scratch, 1,
-               out + row * D, lse ? lse + row : nullptr);
+    tree_merge(acc, S, D, static_cast<int>(threadIdx.x), kCombineThreads, scratch,
+               kCombineScratch, 1, out + row * D, lse ? lse + row : nullptr);
 }
 
 }  // namespace

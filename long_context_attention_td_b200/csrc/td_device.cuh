@@ -165,147 +165,6 @@ struct Elem<__half> {
     }
 };
 
-// ------------------------------------------------------------- row math
-//
-// The consumer keeps q as the raw input elements and forms q.k as an fp32 sum
-// of exact products; the D^-1/2 log2(e) scale is applied to the finished sum.
-// Accumulators of p.v are fp32 pairs in 64-bit registers.  With
-// TD_PACKED_MATH (default) bf16/fp16 products are taken by the mixed-precision
-// fma.rn.f32.{bf16,f16} (no conversion of k) and p.v by fma.rn.f32x2; the
-// alternative converts every element to fp32 first.  The two give identical
-// bits: a bf16 or fp16 product is exact in fp32.
-#ifndef TD_PACKED_MATH
-#define TD_PACKED_MATH 1
-#endif
-
-__device__ __forceinline__ uint64_t pack2(float a, float b) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-    return r;
-}
-
-__device__ __forceinline__ float2 unpack2(uint64_t r) {
-    float2 f;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(r));
-    return f;
-}
-
-// d = a * b + c on two fp32 lanes
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-#if TD_PACKED_MATH
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-#else
-    const float2 x = unpack2(a), y = unpack2(b), z = unpack2(c);
-    return pack2(fmaf(x.x, y.x, z.x), fmaf(x.y, y.y, z.y));
-#endif
-}
-
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-#if TD_PACKED_MATH
-    uint64_t d;
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-#else
-    const float2 x = unpack2(a), y = unpack2(b);
-    return pack2(x.x * y.x, x.y * y.y);
-#endif
-}
-
-template <typename T>
-struct RowMath;
-
-template <>
-struct RowMath<float> {
-    // a += q . k over 4 fp32 elements
-    __device__ __forceinline__ static float dot(const uint4& q, const uint4& k, float a) {
-        a = fmaf(__uint_as_float(q.x), __uint_as_float(k.x), a);
-        a = fmaf(__uint_as_float(q.y), __uint_as_float(k.y), a);
-        a = fmaf(__uint_as_float(q.z), __uint_as_float(k.z), a);
-        a = fmaf(__uint_as_float(q.w), __uint_as_float(k.w), a);
-        return a;
-    }
-    // acc[0..1] += p * v over 4 fp32 elements (pairs)
-    __device__ __forceinline__ static void pv(uint64_t* acc, uint64_t pp, const uint4& v) {
-        acc[0] = fma2(pp, pack2(__uint_as_float(v.x), __uint_as_float(v.y)), acc[0]);
-        acc[1] = fma2(pp, pack2(__uint_as_float(v.z), __uint_as_float(v.w)), acc[1]);
-    }
-};
-
-template <>
-struct RowMath<__nv_bfloat16> {
-    __device__ __forceinline__ static float dot2(uint32_t q, uint32_t k, float a) {
-#if TD_PACKED_MATH
-        asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t"
-            "mov.b32 {ql, qh}, %1;\n\t"
-            "mov.b32 {kl, kh}, %2;\n\t"
-            "fma.rn.f32.bf16 %0, ql, kl, %0;\n\t"
-            "fma.rn.f32.bf16 %0, qh, kh, %0;\n\t}"
-            : "+f"(a)
-            : "r"(q), "r"(k));
-        return a;
-#else
-        a = fmaf(__uint_as_float(q << 16), __uint_as_float(k << 16), a);
-        return fmaf(__uint_as_float(q & 0xffff0000u), __uint_as_float(k & 0xffff0000u), a);
-#endif
-    }
-    __device__ __forceinline__ static float dot(const uint4& q, const uint4& k, float a) {
-        a = dot2(q.x, k.x, a);
-        a = dot2(q.y, k.y, a);
-        a = dot2(q.z, k.z, a);
-        return dot2(q.w, k.w, a);
-    }
-    __device__ __forceinline__ static uint64_t widen(uint32_t w) {
-        return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-    }
-    __device__ __forceinline__ static void pv(uint64_t* acc, uint64_t pp, const uint4& v) {
-        acc[0] = fma2(pp, widen(v.x), acc[0]);
-        acc[1] = fma2(pp, widen(v.y), acc[1]);
-        acc[2] = fma2(pp, widen(v.z), acc[2]);
-        acc[3] = fma2(pp, widen(v.w), acc[3]);
-    }
-};
-
-template <>
-struct RowMath<__half> {
-    __device__ __forceinline__ static float dot2(uint32_t q, uint32_t k, float a) {
-#if TD_PACKED_MATH
-        asm("{\n\t.reg .b16 ql, qh, kl, kh;\n\t"
-            "mov.b32 {ql, qh}, %1;\n\t"
-            "mov.b32 {kl, kh}, %2;\n\t"
-            "fma.rn.f32.f16 %0, ql, kl, %0;\n\t"
-            "fma.rn.f32.f16 %0, qh, kh, %0;\n\t}"
-            : "+f"(a)
-            : "r"(q), "r"(k));
-        return a;
-#else
-        float fq[2], fk[2];
-        Elem<__half>::pair(q, fq);
-        Elem<__half>::pair(k, fk);
-        a = fmaf(fq[0], fk[0], a);
-        return fmaf(fq[1], fk[1], a);
-#endif
-    }
-    __device__ __forceinline__ static float dot(const uint4& q, const uint4& k, float a) {
-        a = dot2(q.x, k.x, a);
-        a = dot2(q.y, k.y, a);
-        a = dot2(q.z, k.z, a);
-        return dot2(q.w, k.w, a);
-    }
-    __device__ __forceinline__ static uint64_t widen(uint32_t w) {
-        float f[2];
-        Elem<__half>::pair(w, f);
-        return pack2(f[0], f[1]);
-    }
-    __device__ __forceinline__ static void pv(uint64_t* acc, uint64_t pp, const uint4& v) {
-        acc[0] = fma2(pp, widen(v.x), acc[0]);
-        acc[1] = fma2(pp, widen(v.y), acc[1]);
-        acc[2] = fma2(pp, widen(v.z), acc[2]);
-        acc[3] = fma2(pp, widen(v.w), acc[3]);
-    }
-};
-
 __device__ __forceinline__ uint4 lds128(const void* p) {
     uint4 r;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -353,29 +212,72 @@ __device__ __forceinline__ float block_sum(float x, int t, int nthreads, float* 
 // num[D]) into out[D] = sum_i e^(m_i - M) num_i / sum_i e^(m_i - M) l_i and
 // lse = (M + log2 L) ln 2, with M = max_i m_i: the gist's global max,
 // renormalisation and sums.  Parts with m = -inf contribute nothing; if all do,
-// out = 0 and lse = -inf.  The sum over parts is split across thread lanes
-// and finished by a pairwise tree in shared memory.
-// `scratch` needs >= nthreads floats.
+// out = 0 and lse = -inf.
+// The parts are taken in chunks: the weights e^(m_i - M) of a chunk are
+// computed once into shared memory, then every thread streams its column
+// slice of the chunk's records with independent loads.  The sum over parts is
+// split across SL thread lanes per column and finished by a pairwise tree, so
+// the order of operations is fixed.  `scratch` holds `scratch_floats` >=
+// nthreads floats.
 template <class Acc>
 __device__ void tree_merge(const Acc& acc, int n, int D, int t, int nthreads, float* scratch,
-                           int bar, float* out_row, float* lse_ptr) {
+                           int scratch_floats, int bar, float* out_row, float* lse_ptr) {
     float mx = kNegInf;
     for (int i = t; i < n; i += nthreads) mx = fmaxf(mx, acc.m2(i));
     const float M = block_max(mx, t, nthreads, scratch, bar);
-    float ls = 0.f;
-    if (M != kNegInf)
-        for (int i = t; i < n; i += nthreads) ls += rescale(acc.m2(i), M) * acc.l(i);
-    const float L = block_sum(ls, t, nthreads, scratch, bar);
 
-    const int DL = D < nthreads ? D : nthreads;
-    int SL = 1;
+    const int DL = D < nthreads ? D : nthreads;  // columns handled at once
+    int SL = 1;                                   // part lanes per column
     while (SL * 2 * DL <= nthreads) SL *= 2;
     const int sl = t / DL, dd = t - sl * DL;
-    for (int d0 = 0; d0 < D; d0 += DL) {
-        const int d = d0 + dd;
-        float a = 0.f;
-        if (sl < SL && d < D && M != kNegInf)
-            for (int i = sl; i < n; i += SL) a += rescale(acc.m2(i), M) * acc.num(i, d);
+    const int passes = (D + DL - 1) / DL;         // 1 or 2 (D <= 2 * nthreads)
+    float a0 = 0.f, a1 = 0.f, ls = 0.f;
+    if (M != kNegInf) {
+        for (int i0 = 0; i0 < n; i0 += scratch_floats) {
+            const int cnt = n - i0 < scratch_floats ? n - i0 : scratch_floats;
+            for (int i = t; i < cnt; i += nthreads) {
+                const float r = rescale(acc.m2(i0 + i), M);
+                scratch[i] = r;
+                ls += r * acc.l(i0 + i);
+            }
+            named_bar_sync(bar, nthreads);
+            if (sl < SL) {
+                const int d0 = dd, d1 = DL + dd;
+                int i = sl;
+#pragma unroll 1
+                for (; i + 3 * SL < cnt; i += 4 * SL) {
+                    const float r0 = scratch[i], r1 = scratch[i + SL];
+                    const float r2 = scratch[i + 2 * SL], r3 = scratch[i + 3 * SL];
+                    const float n0 = acc.num(i0 + i, d0), n1 = acc.num(i0 + i + SL, d0);
+                    const float n2 = acc.num(i0 + i + 2 * SL, d0);
+                    const float n3 = acc.num(i0 + i + 3 * SL, d0);
+                    a0 = fmaf(r0, n0, a0);
+                    a0 = fmaf(r1, n1, a0);
+                    a0 = fmaf(r2, n2, a0);
+                    a0 = fmaf(r3, n3, a0);
+                    if (passes > 1 && d1 < D) {
+                        const float m0 = acc.num(i0 + i, d1), m1 = acc.num(i0 + i + SL, d1);
+                        const float m2v = acc.num(i0 + i + 2 * SL, d1);
+                        const float m3 = acc.num(i0 + i + 3 * SL, d1);
+                        a1 = fmaf(r0, m0, a1);
+                        a1 = fmaf(r1, m1, a1);
+                        a1 = fmaf(r2, m2v, a1);
+                        a1 = fmaf(r3, m3, a1);
+                    }
+                }
+                for (; i < cnt; i += SL) {
+                    const float r = scratch[i];
+                    if (d0 < D) a0 = fmaf(r, acc.num(i0 + i, d0), a0);
+                    if (passes > 1 && d1 < D) a1 = fmaf(r, acc.num(i0 + i, d1), a1);
+                }
+            }
+            named_bar_sync(bar, nthreads);
+        }
+    }
+    const float L = block_sum(ls, t, nthreads, scratch, bar);
+    for (int ps = 0; ps < passes; ++ps) {
+        const float a = ps == 0 ? a0 : a1;
+        const int d = ps * DL + dd;
         if (sl < SL) scratch[sl * DL + dd] = a;
         named_bar_sync(bar, nthreads);
         for (int w = SL >> 1; w > 0; w >>= 1) {

@@ -16,13 +16,13 @@ enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
 #define TD_CONSUMER_WARPS 8
 #endif
 #ifndef TD_STAGES
-#define TD_STAGES 4
+#define TD_STAGES 2
 #endif
 #ifndef TD_STAGE_BYTES
 #define TD_STAGE_BYTES 32768
 #endif
 #ifndef TD_CTAS_PER_SM
-#define TD_CTAS_PER_SM 1
+#define TD_CTAS_PER_SM 3
 #endif
 
 // Consumer warps per CTA of the split-KV kernel, plus one producer warp.

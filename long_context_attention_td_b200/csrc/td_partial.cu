@@ -298,25 +298,27 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         const bool whole = (j0 == 0 && j1 == w.len);
         const long long bh = static_cast<long long>(w.b) * p.H + w.h;
 
-        // q stays in its input element type; the scale goes on the finished sum
-        uint4 qv[C::kNV];
+        // q widened to fp32 once per piece; the D^-1/2 log2(e) scale is applied
+        // to the finished dot product
+        float qf[C::kNV][C::kVec];
         {
             const E* qrow = static_cast<const E*>(p.q) + bh * D;
 #pragma unroll
             for (int u = 0; u < C::kNV; ++u)
-                qv[u] = __ldg(reinterpret_cast<const uint4*>(qrow + (u * C::kG + lig) * C::kVec));
+                Elem<E>::to_f32(
+                    __ldg(reinterpret_cast<const uint4*>(qrow + (u * C::kG + lig) * C::kVec)),
+                    qf[u]);
         }
         const float qscale2 = p.qscale2;
         const bool has_bias = p.slopes != nullptr;
         const float slope2 = has_bias ? __ldg(p.slopes + w.h) * kLog2e : 0.f;
 
-        constexpr int kPairs = C::kVec / 2;  // fp32 pairs per 16-byte vector
         float m = kNegInf, l = 0.f;
-        uint64_t acc[C::kNV][kPairs];
+        float acc[C::kNV][C::kVec];
 #pragma unroll
         for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-            for (int x = 0; x < kPairs; ++x) acc[u][x] = 0ull;
+            for (int x = 0; x < C::kVec; ++x) acc[u][x] = 0.f;
 
         for (long long t0 = j0; t0 < j1; t0 += C::kTile) {
             const long long left = j1 - t0;
@@ -334,9 +336,13 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 float a = 0.f;
                 if (row < rows) {
 #pragma unroll
-                    for (int u = 0; u < C::kNV; ++u)
-                        a = RowMath<E>::dot(
-                            qv[u], lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16), a);
+                    for (int u = 0; u < C::kNV; ++u) {
+                        float kf[C::kVec];
+                        Elem<E>::to_f32(lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16),
+                                        kf);
+#pragma unroll
+                        for (int x = 0; x < C::kVec; ++x) a = fmaf(qf[u][x], kf[x], a);
+                    }
                 }
                 s[i] = a;
             }
@@ -362,22 +368,24 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 const float mn = fmaxf(m, tmax);
                 const float alpha = rescale(m, mn);
                 l *= alpha;
-                const uint64_t aa = pack2(alpha, alpha);
 #pragma unroll
                 for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-                    for (int x = 0; x < kPairs; ++x) acc[u][x] = mul2(acc[u][x], aa);
+                    for (int x = 0; x < C::kVec; ++x) acc[u][x] *= alpha;
 #pragma unroll
                 for (int i = 0; i < C::kRPG; ++i) {
                     const int row = gi + i * C::kNG;
                     if (row < rows) {
                         const float pr = ex2(s[i] - mn);
                         l += pr;
-                        const uint64_t pp = pack2(pr, pr);
 #pragma unroll
-                        for (int u = 0; u < C::kNV; ++u)
-                            RowMath<E>::pv(acc[u], pp,
-                                           lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16));
+                        for (int u = 0; u < C::kNV; ++u) {
+                            float vf[C::kVec];
+                            Elem<E>::to_f32(
+                                lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16), vf);
+#pragma unroll
+                            for (int x = 0; x < C::kVec; ++x) acc[u][x] = fmaf(pr, vf[x], acc[u][x]);
+                        }
                     }
                 }
                 m = mn;
@@ -391,15 +399,6 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         }
 
         // ---- end of piece: merge the row groups of the warp (xor butterfly)
-        float accf[C::kNV][C::kVec];
-#pragma unroll
-        for (int u = 0; u < C::kNV; ++u)
-#pragma unroll
-            for (int x = 0; x < kPairs; ++x) {
-                const float2 f = unpack2(acc[u][x]);
-                accf[u][2 * x] = f.x;
-                accf[u][2 * x + 1] = f.y;
-            }
 #pragma unroll
         for (int o = C::kG; o < 32; o <<= 1) {
             const float mo = __shfl_xor_sync(0xffffffffu, m, o);
@@ -411,8 +410,8 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
                 for (int x = 0; x < C::kVec; ++x) {
-                    const float ao = __shfl_xor_sync(0xffffffffu, accf[u][x], o);
-                    accf[u][x] = accf[u][x] * a + ao * b;
+                    const float ao = __shfl_xor_sync(0xffffffffu, acc[u][x], o);
+                    acc[u][x] = acc[u][x] * a + ao * b;
                 }
             m = M;
         }
@@ -421,7 +420,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
 #pragma unroll
             for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-                for (int x = 0; x < C::kVec; ++x) rw[(u * C::kG + lig) * C::kVec + x] = accf[u][x];
+                for (int x = 0; x < C::kVec; ++x) rw[(u * C::kG + lig) * C::kVec + x] = acc[u][x];
             if (lane == 0) {
                 rw[D] = m;
                 rw[D + 1] = l;
@@ -477,8 +476,8 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             if (ctl.last) {
                 __threadfence();
                 const SlotAcc sa{p.part, c_lo, part_start(c_lo, T, P) < w.start ? 1 : 0, D};
-                tree_merge(sa, n, D, tid, kConsumerThreads, red, kBarConsumers, p.out + bh * D,
-                           p.lse ? p.lse + bh : nullptr);
+                tree_merge(sa, n, D, tid, kConsumerThreads, red, kConsumerWarps * (D + 2),
+                           kBarConsumers, p.out + bh * D, p.lse ? p.lse + bh : nullptr);
             }
             named_bar_sync(kBarConsumers, kConsumerThreads);
         }

@@ -97,7 +97,7 @@ def test_combine_rejects_bad_arguments(L):
     assert L.td_combine(None, f, f, f, None, 1, 1, 4, 128, None) == INVALID
     assert L.td_combine(f, f, f, f, None, 1, 1, 0, 128, None) == INVALID
     assert L.td_combine(f, f, f, f, None, 1, 1, 4, 0, None) == INVALID
-    assert L.td_combine(f, f, f, f, None, 1, 1, 4, 2048, None) == INVALID
+    assert L.td_combine(f, f, f, f, None, 1, 1, 4, 513, None) == INVALID
     assert L.td_combine(f, f, f + 1, f, None, 1, 1, 4, 128, None) == INVALID
 
 
@@ -113,6 +113,7 @@ def test_auto_split_fills_the_gpu_and_respects_part_size(L):
     for (B, H, N) in ((1, 32, 131072), (8, 32, 32768), (1, 8, 1 << 20), (1, 1, 1 << 22)):
         P = L.td_auto_split(B, H, N, 128, 1, sms)
         assert P % sms == 0 and P >= sms
+        assert L.td_auto_split(B, H, N, 128, 1, 2 * sms) == 2 * P
     # tiny problem: no part below 64 KiB of K+V, never more parts than keys
     P = L.td_auto_split(1, 1, 4096, 512, 0, sms)  # fp32 D=512: 4 KiB per key
     assert P == min(sms * (P // sms or 1), 4096 * 4096 // 65536) or P <= 256
