@@ -250,7 +250,7 @@ td_status decode_impl(const Req& r) {
     p.err = reinterpret_cast<int*>(base);
     p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
     p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BH));
-    return cuda_status(td::launch_partial(r.dtype, r.D, p, r.stream));
+    return cuda_status(td::launch_partial(dev, r.dtype, r.D, p, r.stream));
 }
 
 }  // namespace

@@ -243,32 +243,29 @@ __device__ void tree_merge(const Acc& acc, int n, int D, int t, int nthreads, fl
             named_bar_sync(bar, nthreads);
             if (sl < SL) {
                 const int d0 = dd, d1 = DL + dd;
+                const bool two = passes > 1 && d1 < D;
+                constexpr int kBatch = 8;  // independent record loads in flight per thread
                 int i = sl;
 #pragma unroll 1
-                for (; i + 3 * SL < cnt; i += 4 * SL) {
-                    const float r0 = scratch[i], r1 = scratch[i + SL];
-                    const float r2 = scratch[i + 2 * SL], r3 = scratch[i + 3 * SL];
-                    const float n0 = acc.num(i0 + i, d0), n1 = acc.num(i0 + i + SL, d0);
-                    const float n2 = acc.num(i0 + i + 2 * SL, d0);
-                    const float n3 = acc.num(i0 + i + 3 * SL, d0);
-                    a0 = fmaf(r0, n0, a0);
-                    a0 = fmaf(r1, n1, a0);
-                    a0 = fmaf(r2, n2, a0);
-                    a0 = fmaf(r3, n3, a0);
-                    if (passes > 1 && d1 < D) {
-                        const float m0 = acc.num(i0 + i, d1), m1 = acc.num(i0 + i + SL, d1);
-                        const float m2v = acc.num(i0 + i + 2 * SL, d1);
-                        const float m3 = acc.num(i0 + i + 3 * SL, d1);
-                        a1 = fmaf(r0, m0, a1);
-                        a1 = fmaf(r1, m1, a1);
-                        a1 = fmaf(r2, m2v, a1);
-                        a1 = fmaf(r3, m3, a1);
+                for (; i + (kBatch - 1) * SL < cnt; i += kBatch * SL) {
+                    float x0[kBatch], x1[kBatch];
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) x0[j] = acc.num(i0 + i + j * SL, d0);
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < kBatch; ++j) x1[j] = acc.num(i0 + i + j * SL, d1);
+                    }
+#pragma unroll
+                    for (int j = 0; j < kBatch; ++j) a0 = fmaf(scratch[i + j * SL], x0[j], a0);
+                    if (two) {
+#pragma unroll
+                        for (int j = 0; j < kBatch; ++j) a1 = fmaf(scratch[i + j * SL], x1[j], a1);
                     }
                 }
                 for (; i < cnt; i += SL) {
                     const float r = scratch[i];
                     if (d0 < D) a0 = fmaf(r, acc.num(i0 + i, d0), a0);
-                    if (passes > 1 && d1 < D) a1 = fmaf(r, acc.num(i0 + i, d1), a1);
+                    if (two) a1 = fmaf(r, acc.num(i0 + i, d1), a1);
                 }
             }
             named_bar_sync(bar, nthreads);

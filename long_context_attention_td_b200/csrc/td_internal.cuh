@@ -65,8 +65,9 @@ size_t partial_smem_bytes(int dtype, int D);
 // CTAs of the split-KV kernel that fit on one SM (static estimate from shared
 // memory and threads; matches the kernel's launch bounds).
 int partial_ctas_per_sm(int dtype, int D);
-// Launch the split-KV kernel (grid = p.P) with its fused combine.
-cudaError_t launch_partial(int dtype, int D, const PartialParams& p, cudaStream_t s);
+// Launch the split-KV kernel (grid = p.P) with its fused combine on `device`
+// (the current device).
+cudaError_t launch_partial(int device, int dtype, int D, const PartialParams& p, cudaStream_t s);
 // Launch the standalone tree combine over dense partials.
 cudaError_t launch_combine(const float* num, const float* m, const float* l, float* out,
                            float* lse, int64_t rows, int S, int D, cudaStream_t s);

@@ -23,6 +23,8 @@
 // Warps 0-7 consume: a group of kG lanes owns one key row per step, each lane
 // holding 16 bytes of q, k, v and its slice of the fp32 accumulator; the dot
 // product is finished with xor shuffles inside the group.
+#include <atomic>
+
 #include "td_device.cuh"
 #include "td_internal.cuh"
 #include "treedec.h"
@@ -486,23 +488,29 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
 }
 
 template <typename T, int D>
-cudaError_t launch_t(const PartialParams& p, cudaStream_t s) {
+cudaError_t launch_t(int device, const PartialParams& p, cudaStream_t s) {
     using C = Cfg<T, D>;
     auto kern = td_partial_kernel<T, D>;
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem));
-    if (e != cudaSuccess) return e;
+    // the dynamic shared-memory opt-in is per device: set it once on each
+    static std::atomic<unsigned long long> configured{0};
+    const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
+    if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem));
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
     kern<<<static_cast<unsigned>(p.P), kPartialThreads, C::kSmem, s>>>(p);
     return cudaGetLastError();
 }
 
 template <typename T>
-cudaError_t launch_d(int D, const PartialParams& p, cudaStream_t s) {
+cudaError_t launch_d(int device, int D, const PartialParams& p, cudaStream_t s) {
     switch (D) {
-        case 64: return launch_t<T, 64>(p, s);
-        case 128: return launch_t<T, 128>(p, s);
-        case 256: return launch_t<T, 256>(p, s);
-        case 512: return launch_t<T, 512>(p, s);
+        case 64: return launch_t<T, 64>(device, p, s);
+        case 128: return launch_t<T, 128>(device, p, s);
+        case 256: return launch_t<T, 256>(device, p, s);
+        case 512: return launch_t<T, 512>(device, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -520,11 +528,11 @@ size_t smem_d(int D) {
 
 }  // namespace
 
-cudaError_t launch_partial(int dtype, int D, const PartialParams& p, cudaStream_t s) {
+cudaError_t launch_partial(int device, int dtype, int D, const PartialParams& p, cudaStream_t s) {
     switch (dtype) {
-        case kF32: return launch_d<float>(D, p, s);
-        case kBF16: return launch_d<__nv_bfloat16>(D, p, s);
-        case kF16: return launch_d<__half>(D, p, s);
+        case kF32: return launch_d<float>(device, D, p, s);
+        case kBF16: return launch_d<__nv_bfloat16>(device, D, p, s);
+        case kF16: return launch_d<__half>(device, D, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
