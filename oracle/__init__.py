@@ -55,6 +55,10 @@ def lib():
         L.or_full.argtypes = common + [vp, vp, ctypes.c_int]
         L.or_chunked.restype = ctypes.c_int
         L.or_chunked.argtypes = common + [ctypes.c_int, ctypes.c_int, vp, vp, ctypes.c_int]
+        L.or_full_gqa.restype = ctypes.c_int
+        L.or_full_gqa.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                  ctypes.c_int, ctypes.c_int64, ctypes.c_int, vp, vp, vp,
+                                  ctypes.c_int64, vp, vp, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -121,6 +125,30 @@ def full(q, k, v, slopes=None, seqlens=None, bh=None, threads=0):
     (out [n_bh, D], lse [n_bh]), lse the absolute natural-log log-sum-exp.
     """
     return _batched("or_full", q, k, v, slopes, seqlens, bh, threads)
+
+
+def full_gqa(q, k, v, slopes=None, seqlens=None, bh=None, threads=0):
+    """Grouped-query plain decode: q [B,H,1,D], k/v [B,Hkv,N,D] with H a
+    multiple of Hkv (query head h reads kv head h // (H // Hkv)); slopes [H].
+    Returns (out [n_bh, D], lse [n_bh]) over the listed b*H+h (all by default)."""
+    cq, tq, pq = _code_and_buf(q)
+    ck, tk, pk = _code_and_buf(k)
+    cv, tv, pv = _code_and_buf(v)
+    if not (cq == ck == cv):
+        raise TypeError("q, k, v must share one element type")
+    B, H, _, D = tuple(tq.shape)
+    Hkv, Nmax = int(tk.shape[1]), int(tk.shape[2])
+    if tuple(tk.shape) != (B, Hkv, Nmax, D) or tuple(tv.shape) != (B, Hkv, Nmax, D):
+        raise ValueError("layout must be q[B,H,1,D], k/v[B,Hkv,N,D]")
+    sl = None if slopes is None else np.ascontiguousarray(np.asarray(slopes, dtype=np.float32))
+    sq = None if seqlens is None else np.ascontiguousarray(np.asarray(seqlens, dtype=np.int32))
+    bl = None if bh is None else np.ascontiguousarray(np.asarray(bh, dtype=np.int64))
+    n_bh = B * H if bl is None else len(bl)
+    out = np.zeros((n_bh, D), dtype=np.float64)
+    lse = np.zeros((n_bh,), dtype=np.float64)
+    _check(lib().or_full_gqa(pq, pk, pv, cq, B, H, Hkv, Nmax, D, _ptr(sq), _ptr(sl), _ptr(bl),
+                             n_bh, out.ctypes.data, lse.ctypes.data, int(threads)), "full_gqa")
+    return out, lse
 
 
 def chunked(q, k, v, n_chunks, mode="torch_chunk", slopes=None, seqlens=None, bh=None,

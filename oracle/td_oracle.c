@@ -295,6 +295,7 @@ static int attend_chunked(const void *q, int64_t q_off, const void *k, const voi
 typedef struct {
     const void *q, *k, *v;
     int dtype, B, H, D;
+    int Hkv;                /* key/value heads; query head h reads kv head h / (H / Hkv) */
     int64_t Nmax;
     const int32_t *seqlens; /* host, [B], or NULL: every sequence has Nmax keys */
     const float *slopes;    /* host, [H], or NULL: no bias */
@@ -313,10 +314,11 @@ static void *worker(void *arg) {
         if (i >= J->n_bh) break;
         int64_t bh = J->bh ? J->bh[i] : i;
         int64_t b = bh / J->H, h = bh % J->H;
+        int64_t hkv = h / (J->H / J->Hkv);
         int64_t n = J->seqlens ? (int64_t)J->seqlens[b] : J->Nmax;
         double slope = J->slopes ? (double)J->slopes[h] : 0.0;
         int64_t q_off = bh * (int64_t)J->D;
-        int64_t kv_off = bh * J->Nmax * (int64_t)J->D;
+        int64_t kv_off = (b * J->Hkv + hkv) * J->Nmax * (int64_t)J->D;
         int rc;
         if (J->chunks == 0)
             rc = attend(J->q, q_off, J->k, J->v, kv_off, J->dtype, J->D, n, slope, NULL,
@@ -332,7 +334,7 @@ static void *worker(void *arg) {
 static int run(job_t *J, int threads) {
     if (!J->q || !J->k || !J->v || !J->out || !J->lse) return -1;
     if (J->dtype < OR_F32 || J->dtype > OR_F16 || J->B <= 0 || J->H <= 0 || J->D <= 0 ||
-        J->Nmax < 0 || J->n_bh < 0)
+        J->Nmax < 0 || J->n_bh < 0 || J->Hkv <= 0 || J->H % J->Hkv != 0)
         return -1;
     if (J->seqlens)
         for (int b = 0; b < J->B; ++b)
@@ -364,7 +366,22 @@ static int run(job_t *J, int threads) {
 int or_full(const void *q, const void *k, const void *v, int dtype, int B, int H,
             int64_t Nmax, int D, const int32_t *seqlens, const float *slopes,
             const int64_t *bh, int64_t n_bh, double *out, double *lse, int threads) {
-    job_t J = {q, k, v, dtype, B, H, D, Nmax, seqlens, slopes, bh,
+    job_t J = {q, k, v, dtype, B, H, D, H, Nmax, seqlens, slopes, bh,
+               bh ? n_bh : (int64_t)B * H, 0, 0, out, lse, 0, 0};
+    return run(&J, threads);
+}
+
+/*
+ * Grouped-query form of the plain definition: H query heads share Hkv
+ * key/value heads (H a multiple of Hkv), query head h attending to kv head
+ * h / (H / Hkv).  Layout q [B,H,1,D], k/v [B,Hkv,Nmax,D]; slopes per query
+ * head [H]; bh lists b*H+h over query heads.  Hkv = 1 is multi-query
+ * attention, Hkv = H is or_full.
+ */
+int or_full_gqa(const void *q, const void *k, const void *v, int dtype, int B, int H, int Hkv,
+                int64_t Nmax, int D, const int32_t *seqlens, const float *slopes,
+                const int64_t *bh, int64_t n_bh, double *out, double *lse, int threads) {
+    job_t J = {q, k, v, dtype, B, H, D, Hkv, Nmax, seqlens, slopes, bh,
                bh ? n_bh : (int64_t)B * H, 0, 0, out, lse, 0, 0};
     return run(&J, threads);
 }
@@ -375,7 +392,7 @@ int or_chunked(const void *q, const void *k, const void *v, int dtype, int B, in
                const int64_t *bh, int64_t n_bh, int w, int mode, double *out,
                double *lse, int threads) {
     if (w <= 0 || (mode != 0 && mode != 1)) return -1;
-    job_t J = {q, k, v, dtype, B, H, D, Nmax, seqlens, slopes, bh,
+    job_t J = {q, k, v, dtype, B, H, D, H, Nmax, seqlens, slopes, bh,
                bh ? n_bh : (int64_t)B * H, w, mode, out, lse, 0, 0};
     return run(&J, threads);
 }

@@ -411,3 +411,35 @@ def test_threads_do_not_change_results():
     o8, l8 = oracle.full(q, k, v, threads=8)
     np.testing.assert_array_equal(o1, o8)
     np.testing.assert_array_equal(l1, l8)
+
+
+# ------------------------------------------------------- grouped-query form
+
+@pytest.mark.parametrize("H,Hkv", [(8, 1), (8, 2), (8, 8), (6, 3)])
+def test_gqa_equals_mha_on_repeated_kv(H, Hkv):
+    """Grouped-query attention is plain attention with each kv head repeated
+    for the query heads that share it."""
+    B, N, D = 2, 37, 16
+    q = _rand((B, H, 1, D), torch.bfloat16, 161)
+    k = _rand((B, Hkv, N, D), torch.bfloat16, 162)
+    v = _rand((B, Hkv, N, D), torch.bfloat16, 163)
+    slopes = torch.linspace(0.05, 0.9, H).float()
+    seqlens = [20, 37]
+    o, l = oracle.full_gqa(q, k, v, slopes=slopes, seqlens=seqlens)
+    G = H // Hkv
+    kr = k.repeat_interleave(G, dim=1).contiguous()
+    vr = v.repeat_interleave(G, dim=1).contiguous()
+    ro, rl = oracle.full(q, kr, vr, slopes=slopes, seqlens=seqlens)
+    np.testing.assert_array_equal(o, ro)
+    np.testing.assert_array_equal(l, rl)
+
+
+def test_gqa_vs_torch_sdpa_enable_gqa():
+    B, H, Hkv, N, D = 1, 8, 2, 29, 32
+    q = _rand((B, H, 1, D), torch.float32, 171)
+    k = _rand((B, Hkv, N, D), torch.float32, 172)
+    v = _rand((B, Hkv, N, D), torch.float32, 173)
+    o, l = oracle.full_gqa(q, k, v)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.double(), k.double(), v.double(), enable_gqa=True)
+    np.testing.assert_allclose(o, ref.reshape(B * H, D).numpy(), rtol=0, atol=1e-12)
