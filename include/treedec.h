@@ -133,6 +133,45 @@ TD_API td_status td_decode_ws(const void *q, const void *k, const void *v, float
                        size_t workspace_bytes, td_stream stream);
 
 /*
+ * td_decode_gqa -- grouped-query (and multi-query) decode: Hq query heads
+ * share Hkv key/value heads, query head h attending to kv head h / (Hq/Hkv)
+ * (the pages' per-head decode with the key/value tile shared by the G =
+ * Hq/Hkv queries of a group; Hkv = 1 is multi-query attention).  Each K/V
+ * tile is read once for its G queries and the two products S = Q K^T and
+ * P V run on the tensor cores (tcgen05), with fp32 accumulation; p is rounded
+ * to the input element type before P V (error ~2^-9 relative for bf16).
+ *   q        device [B,Hq,1,D]; k, v device [B,Hkv,N,D] (padded Nmax when
+ *            seqlens is given); dtype TD_BF16 or TD_F16; D 64 or 128;
+ *            1 <= Hq/Hkv <= 128; B*Hkv*N < 2^31.
+ *   out      device fp32 [B,Hq,1,D]; lse device fp32 [B,Hq,1] or NULL.
+ *   seqlens / seqlens_host  as td_decode_varlen, or both NULL.
+ *   n_split  0: heuristic; > 0: parts per (b, kv head) (equal lengths), or
+ *            B*Hkv*n_split parts over the flattened keys (ragged).
+ *   alibi_slopes  device fp32 [Hq] (per query head) or NULL.
+ */
+TD_API td_status td_decode_gqa(const void *q, const void *k, const void *v, float *out, float *lse,
+                               int B, int Hq, int Hkv, int64_t N, int D, const int32_t *seqlens,
+                               const int32_t *seqlens_host, int n_split,
+                               const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
+/* td_decode_gqa with a caller-owned workspace (td_gqa_workspace_bytes) and an
+ * explicit part count over the flattened (b, kv head, key) space (0 =
+ * heuristic: td_plan_parts_gqa); same workspace rules as td_decode_ws. */
+TD_API td_status td_decode_gqa_ws(const void *q, const void *k, const void *v, float *out,
+                                  float *lse, int B, int Hq, int Hkv, int64_t N, int D,
+                                  const int32_t *seqlens, const int32_t *seqlens_host,
+                                  int64_t parts, const float *alibi_slopes, td_dtype dtype,
+                                  void *workspace, size_t workspace_bytes, td_stream stream);
+
+/* Part count td_decode_gqa would use on the current device (total_keys as in
+ * td_plan_parts: < 0 for equal lengths Nmax); -1 on invalid arguments. */
+TD_API int64_t td_plan_parts_gqa(int B, int Hq, int Hkv, int64_t Nmax, int D, td_dtype dtype,
+                                 int n_split, int64_t total_keys);
+
+/* Bytes of workspace td_decode_gqa_ws needs for `parts` parts. */
+TD_API size_t td_gqa_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t parts);
+
+/*
  * td_combine -- merge caller-provided partials into the final output: the
  * gist's global max, renormalisation and two sums (tree_attn_decode after
  * "first get global max"), done per (b,h) as a log-depth tree on the GPU.

@@ -19,7 +19,8 @@ import torch
 __all__ = [
     "TreeDecError", "lib", "library_path", "decode", "decode_varlen", "decode_ws", "combine",
     "auto_split", "plan_parts", "workspace_bytes", "decode_host", "check_device_error",
-    "release_workspace", "DTYPE_CODE",
+    "release_workspace", "DTYPE_CODE", "decode_gqa", "decode_gqa_ws", "plan_parts_gqa",
+    "gqa_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +63,16 @@ def lib():
     L.td_decode_ws.restype = i32
     L.td_decode_ws.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp, i64, vp, i32,
                                vp, sz, vp]
+    L.td_decode_gqa.restype = i32
+    L.td_decode_gqa.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp, i32, vp,
+                                i32, vp]
+    L.td_decode_gqa_ws.restype = i32
+    L.td_decode_gqa_ws.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, i32, vp, vp, i64, vp,
+                                   i32, vp, sz, vp]
+    L.td_plan_parts_gqa.restype = i64
+    L.td_plan_parts_gqa.argtypes = [i32, i32, i32, i64, i32, i32, i32, i64]
+    L.td_gqa_workspace_bytes.restype = sz
+    L.td_gqa_workspace_bytes.argtypes = [i32, i32, i32, i32, i64]
     L.td_combine.restype = i32
     L.td_combine.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, vp]
     L.td_auto_split.restype = i64
@@ -191,6 +202,65 @@ def decode_ws(q, k, v, workspace, *, seqlens=None, seqlens_host=None, parts=0, s
                             DTYPE_CODE[q.dtype], _ptr(workspace), nbytes, _stream(stream))
     _check(st, "td_decode_ws")
     return out, lse
+
+
+def _gqa_shapes(q, k, v):
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("expected q [B,Hq,1,D], k and v [B,Hkv,N,D]")
+    B, Hq, one, D = q.shape
+    if one != 1 or k.shape[0] != B or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError("expected q [B,Hq,1,D], k and v [B,Hkv,N,D]")
+    if q.dtype != k.dtype or q.dtype != v.dtype or q.dtype not in DTYPE_CODE:
+        raise TypeError("q, k, v must share one of bfloat16, float16")
+    return B, Hq, int(k.shape[1]), int(k.shape[2]), D
+
+
+def decode_gqa(q, k, v, *, seqlens=None, seqlens_host=None, slopes=None, n_split=0, out=None,
+               lse=None, stream=None):
+    """Grouped-query decode (tensor cores): q [B,Hq,1,D], k/v [B,Hkv,N,D]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev_tensor(t, n)
+    B, Hq, Hkv, N, D = _gqa_shapes(q, k, v)
+    if seqlens is not None:
+        _dev_tensor(seqlens, "seqlens", torch.int32)
+    sh = None if seqlens_host is None else seqlens_host.to(torch.int32).contiguous().cpu()
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    out, lse = _outputs(q, B, Hq, D, out, lse)
+    st = lib().td_decode_gqa(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N, D,
+                             _ptr(seqlens), _ptr(sh), int(n_split), _ptr(slopes),
+                             DTYPE_CODE[q.dtype], _stream(stream))
+    _check(st, "td_decode_gqa")
+    return out, lse
+
+
+def decode_gqa_ws(q, k, v, workspace, *, seqlens=None, seqlens_host=None, parts=0, slopes=None,
+                  out=None, lse=None, stream=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev_tensor(t, n)
+    B, Hq, Hkv, N, D = _gqa_shapes(q, k, v)
+    _dev_tensor(workspace, "workspace")
+    if seqlens is not None:
+        _dev_tensor(seqlens, "seqlens", torch.int32)
+    sh = None if seqlens_host is None else seqlens_host.to(torch.int32).contiguous().cpu()
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    out, lse = _outputs(q, B, Hq, D, out, lse)
+    nbytes = workspace.numel() * workspace.element_size()
+    st = lib().td_decode_gqa_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, N,
+                                D, _ptr(seqlens), _ptr(sh), int(parts), _ptr(slopes),
+                                DTYPE_CODE[q.dtype], _ptr(workspace), nbytes, _stream(stream))
+    _check(st, "td_decode_gqa_ws")
+    return out, lse
+
+
+def plan_parts_gqa(B, Hq, Hkv, Nmax, D, dtype, n_split=0, total_keys=-1):
+    return int(lib().td_plan_parts_gqa(int(B), int(Hq), int(Hkv), int(Nmax), int(D),
+                                       DTYPE_CODE[dtype], int(n_split), int(total_keys)))
+
+
+def gqa_workspace_bytes(B, Hq, Hkv, D, parts):
+    return int(lib().td_gqa_workspace_bytes(int(B), int(Hq), int(Hkv), int(D), int(parts)))
 
 
 def combine(num, m, l, *, out=None, lse=None, stream=None):

@@ -2,6 +2,8 @@
 // per-device workspace and staging buffers, and the extern "C" entry points
 // declared in treedec.h.  Nothing here computes attention: every step of the
 // decode runs in the kernels of td_partial.cu and td_combine.cu.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -147,6 +149,35 @@ td_status library_ws(int dev, size_t need, cudaStream_t stream, void** ws, size_
     return TD_OK;
 }
 
+// The workspace a call runs on: the caller's (checked) or the library's
+// (grown), with its first `tickets` tickets known to be zero.
+td_status prepare_ws(int dev, void* user_ws, size_t user_bytes, long long tickets, size_t need,
+                     cudaStream_t stream, char** base_out) {
+    void* ws = user_ws;
+    size_t wsb = user_bytes;
+    td_status st = TD_OK;
+    if (ws) {
+        if (!aligned(ws, 256)) return TD_ERR_INVALID_ARG;
+        if (wsb < need) return TD_ERR_WORKSPACE;
+    } else {
+        st = library_ws(dev, need, stream, &ws, &wsb);
+        if (st != TD_OK) return st;
+    }
+    char* base = static_cast<char*>(ws);
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        const KnownZero* e = known_entry(ws);
+        if (!e || e->tickets < tickets) {
+            st = cuda_status(
+                cudaMemsetAsync(base + td::kErrRegion, 0, ticket_region(tickets), stream));
+            if (st != TD_OK) return st;
+        }
+        remember_workspace(ws, tickets);
+    }
+    *base_out = base;
+    return TD_OK;
+}
+
 struct Req {
     const void *q, *k, *v;
     float *out, *lse;
@@ -213,26 +244,9 @@ td_status decode_impl(const Req& r) {
     const long long BH = static_cast<long long>(r.B) * r.H;
     if (!mul_fits(P + 1, BH * r.N)) return TD_ERR_INVALID_ARG;
     const size_t need = ws_bytes_for(BH, r.D, P);
-    void* ws = r.ws;
-    size_t wsb = r.ws_bytes;
-    if (ws) {
-        if (!aligned(ws, 256)) return TD_ERR_INVALID_ARG;
-        if (wsb < need) return TD_ERR_WORKSPACE;
-    } else {
-        st = library_ws(dev, need, r.stream, &ws, &wsb);
-        if (st != TD_OK) return st;
-    }
-    char* base = static_cast<char*>(ws);
-    {
-        std::lock_guard<std::mutex> lk(g_mu);
-        const KnownZero* e = known_entry(ws);
-        if (!e || e->tickets < BH) {
-            st = cuda_status(
-                cudaMemsetAsync(base + td::kErrRegion, 0, ticket_region(BH), r.stream));
-            if (st != TD_OK) return st;
-        }
-        remember_workspace(ws, BH);
-    }
+    char* base = nullptr;
+    st = prepare_ws(dev, r.ws, r.ws_bytes, BH, need, r.stream, &base);
+    if (st != TD_OK) return st;
     td::PartialParams p;
     p.q = r.q;
     p.k = r.k;
@@ -253,9 +267,214 @@ td_status decode_impl(const Req& r) {
     return cuda_status(td::launch_partial(dev, r.dtype, r.D, p, r.stream));
 }
 
+// ------------------------------------------------------------- grouped-query
+
+constexpr int kGqaCtasPerSm = 1;
+
+size_t gqa_ws_bytes_for(long long BHkv, int G, int D, long long parts) {
+    return td::kErrRegion + ticket_region(BHkv) +
+           static_cast<size_t>(parts) * 2 * static_cast<size_t>(G) *
+               static_cast<size_t>(D + 3) * sizeof(float);
+}
+
+long long gqa_auto_parts(long long T, int D, int num_sms) {
+    if (T <= 0) return 1;
+    const long long fill = static_cast<long long>(num_sms) * kGqaCtasPerSm;
+    const long long bytes_per_key = 2LL * D * 2;
+    long long by_size = T / (td::kMinPartBytes / bytes_per_key);
+    if (by_size < 1) by_size = 1;
+    long long P = fill < by_size ? fill : by_size;
+    if (P > T) P = T;
+    return P < 1 ? 1 : P;
+}
+
+struct GqaReq {
+    const void *q, *k, *v;
+    float *out, *lse;
+    int B, Hq, Hkv;
+    long long N;
+    int D;
+    const int32_t* seqlens;
+    const int32_t* seqlens_host;
+    long long parts;  // 0 = heuristic
+    int n_split;      // used when parts == 0 and n_split > 0
+    const float* slopes;
+    int dtype;
+    void* ws;
+    size_t ws_bytes;
+    cudaStream_t stream;
+};
+
+td_status gqa_validate(const GqaReq& r) {
+    if (!r.q || !r.k || !r.v || !r.out) return TD_ERR_INVALID_ARG;
+    if (r.dtype != TD_BF16 && r.dtype != TD_F16) return TD_ERR_UNSUPPORTED;
+    if (r.D != 64 && r.D != 128) return TD_ERR_UNSUPPORTED;
+    if (r.B < 1 || r.Hq < 1 || r.Hkv < 1 || r.N < 1 || r.parts < 0 || r.n_split < 0)
+        return TD_ERR_INVALID_ARG;
+    if (r.Hq % r.Hkv != 0) return TD_ERR_INVALID_ARG;
+    if (r.Hq / r.Hkv > 128) return TD_ERR_UNSUPPORTED;
+    if (!aligned(r.q, 16) || !aligned(r.k, 16) || !aligned(r.v, 16)) return TD_ERR_INVALID_ARG;
+    if (!aligned(r.out, 4) || (r.lse && !aligned(r.lse, 4)) ||
+        (r.slopes && !aligned(r.slopes, 4)) || (r.seqlens && !aligned(r.seqlens, 4)))
+        return TD_ERR_INVALID_ARG;
+    if (r.seqlens_host && !r.seqlens) return TD_ERR_INVALID_ARG;
+    const long long BHkv = static_cast<long long>(r.B) * r.Hkv;
+    if (static_cast<long long>(r.B) * r.Hq > 0x7fffffffLL) return TD_ERR_INVALID_ARG;
+    // the tensor-map row coordinate is a 32-bit integer
+    if (!mul_fits(BHkv, r.N) || BHkv * r.N > 0x7fffffffLL) return TD_ERR_INVALID_ARG;
+    if (r.seqlens_host)
+        for (int b = 0; b < r.B; ++b)
+            if (r.seqlens_host[b] < 0 || r.seqlens_host[b] > r.N) return TD_ERR_INVALID_ARG;
+    return TD_OK;
+}
+
+long long gqa_plan(const GqaReq& r, int num_sms) {
+    const long long BHkv = static_cast<long long>(r.B) * r.Hkv;
+    const long long bound = BHkv * r.N;
+    long long known = -1;
+    if (!r.seqlens) {
+        known = bound;
+    } else if (r.seqlens_host) {
+        long long s = 0;
+        for (int b = 0; b < r.B; ++b) s += r.seqlens_host[b];
+        known = s * r.Hkv;
+    }
+    const long long T = known >= 0 ? known : bound;
+    long long P = r.parts;
+    if (P == 0 && r.n_split > 0) {
+        const long long per = (!r.seqlens && r.n_split > r.N) ? r.N : r.n_split;
+        P = BHkv * per;
+    }
+    if (P == 0) P = gqa_auto_parts(T, r.D, num_sms);
+    const long long cap = T > 0 ? T : 1;
+    if (P > cap) P = cap;
+    if (P > 0x7fffffffLL) P = 0x7fffffffLL;
+    return P < 1 ? 1 : P;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D map over [rows, D] elements, box {64 columns, 64 rows}, 128-byte swizzle,
+// out-of-range rows read as zero.
+td_status make_kv_map(CUtensorMap* map, const void* base, long long rows, int D, int dtype) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return TD_ERR_CUDA;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    cuuint32_t box[2] = {64, 64};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult rc = enc(map,
+                            dtype == TD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS ? TD_OK : TD_ERR_INVALID_ARG;
+}
+
+td_status gqa_impl(const GqaReq& r) {
+    td_status st = gqa_validate(r);
+    if (st != TD_OK) return st;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TD_OK) return st;
+    const long long P = gqa_plan(r, sms);
+    const long long BHkv = static_cast<long long>(r.B) * r.Hkv;
+    if (!mul_fits(P + 1, BHkv * r.N)) return TD_ERR_INVALID_ARG;
+    const int G = r.Hq / r.Hkv;
+    const size_t need = gqa_ws_bytes_for(BHkv, G, r.D, P);
+    CUtensorMap mk, mv;
+    st = make_kv_map(&mk, r.k, BHkv * r.N, r.D, r.dtype);
+    if (st != TD_OK) return st;
+    st = make_kv_map(&mv, r.v, BHkv * r.N, r.D, r.dtype);
+    if (st != TD_OK) return st;
+    char* base = nullptr;
+    st = prepare_ws(dev, r.ws, r.ws_bytes, BHkv, need, r.stream, &base);
+    if (st != TD_OK) return st;
+    td::GqaParams p;
+    p.q = r.q;
+    p.out = r.out;
+    p.lse = r.lse;
+    p.slopes = r.slopes;
+    p.seqlens = r.seqlens;
+    p.B = r.B;
+    p.Hq = r.Hq;
+    p.Hkv = r.Hkv;
+    p.G = G;
+    p.N = r.N;
+    p.T = r.seqlens ? -1 : BHkv * r.N;
+    p.P = P;
+    p.qscale2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(r.D)));
+    p.err = reinterpret_cast<int*>(base);
+    p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
+    p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BHkv));
+    return cuda_status(td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
+}
+
 }  // namespace
 
 extern "C" {
+
+td_status td_decode_gqa(const void* q, const void* k, const void* v, float* out, float* lse, int B,
+                        int Hq, int Hkv, int64_t N, int D, const int32_t* seqlens,
+                        const int32_t* seqlens_host, int n_split, const float* alibi_slopes,
+                        td_dtype dtype, td_stream stream) {
+    GqaReq r{q, k, v, out, lse, B, Hq, Hkv, N, D, seqlens, seqlens_host, 0, n_split,
+             alibi_slopes, static_cast<int>(dtype), nullptr, 0,
+             reinterpret_cast<cudaStream_t>(stream)};
+    return gqa_impl(r);
+}
+
+td_status td_decode_gqa_ws(const void* q, const void* k, const void* v, float* out, float* lse,
+                           int B, int Hq, int Hkv, int64_t N, int D, const int32_t* seqlens,
+                           const int32_t* seqlens_host, int64_t parts, const float* alibi_slopes,
+                           td_dtype dtype, void* workspace, size_t workspace_bytes,
+                           td_stream stream) {
+    if (!workspace || parts < 0) return TD_ERR_INVALID_ARG;
+    GqaReq r{q, k, v, out, lse, B, Hq, Hkv, N, D, seqlens, seqlens_host, parts, 0,
+             alibi_slopes, static_cast<int>(dtype), workspace, workspace_bytes,
+             reinterpret_cast<cudaStream_t>(stream)};
+    return gqa_impl(r);
+}
+
+int64_t td_plan_parts_gqa(int B, int Hq, int Hkv, int64_t Nmax, int D, td_dtype dtype,
+                          int n_split, int64_t total_keys) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Nmax < 1 || n_split < 0 || Hq % Hkv != 0) return -1;
+    if ((dtype != TD_BF16 && dtype != TD_F16) || (D != 64 && D != 128)) return -1;
+    const long long BHkv = static_cast<long long>(B) * Hkv;
+    if (!mul_fits(BHkv, Nmax) || (total_keys >= 0 && total_keys > BHkv * Nmax)) return -1;
+    int dev = 0, sms = 0;
+    if (current_device(&dev, &sms) != TD_OK) return -1;
+    GqaReq r{nullptr, nullptr, nullptr, nullptr, nullptr, B, Hq, Hkv, Nmax, D, nullptr, nullptr,
+             0, n_split, nullptr, static_cast<int>(dtype), nullptr, 0, nullptr};
+    if (total_keys >= 0) {
+        // ragged: size from the given key count
+        long long T = total_keys;
+        long long P = n_split > 0 ? BHkv * n_split : gqa_auto_parts(T, D, sms);
+        const long long cap = T > 0 ? T : 1;
+        if (P > cap) P = cap;
+        return P < 1 ? 1 : P;
+    }
+    return gqa_plan(r, sms);
+}
+
+size_t td_gqa_workspace_bytes(int B, int Hq, int Hkv, int D, int64_t parts) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || D < 1 || parts < 1) return 0;
+    return gqa_ws_bytes_for(static_cast<long long>(B) * Hkv, Hq / Hkv, D, parts);
+}
+
 
 td_status td_decode(const void* q, const void* k, const void* v, float* out, float* lse, int B,
                     int H, int64_t N, int D, int n_split, const float* alibi_slopes,

@@ -18,6 +18,7 @@ constexpr int kCombineScratch = 2048;  // weights of up to 2048 parts per chunk
 // Dense caller layout: num [rows, S, D], m and l [rows, S], m in natural-log
 // units (converted to the log2 units of tree_merge).
 struct DenseAcc {
+    static constexpr bool kSplitL = false;
     const float* pn;
     const float* pm;
     const float* pl;

@@ -272,6 +272,15 @@ __device__ void tree_merge(const Acc& acc, int n, int D, int t, int nthreads, fl
         }
     }
     const float L = block_sum(ls, t, nthreads, scratch, bar);
+    // parts may carry a second denominator for the lse (sum of unrounded p when
+    // the numerator was formed with rounded p)
+    float Lx = L;
+    if constexpr (Acc::kSplitL) {
+        float lx = 0.f;
+        if (M != kNegInf)
+            for (int i = t; i < n; i += nthreads) lx += rescale(acc.m2(i), M) * acc.lx(i);
+        Lx = block_sum(lx, t, nthreads, scratch, bar);
+    }
     for (int ps = 0; ps < passes; ++ps) {
         const float a = ps == 0 ? a0 : a1;
         const int d = ps * DL + dd;
@@ -284,7 +293,7 @@ __device__ void tree_merge(const Acc& acc, int n, int D, int t, int nthreads, fl
         if (sl == 0 && d < D) out_row[d] = M == kNegInf ? 0.f : scratch[dd] / L;
         named_bar_sync(bar, nthreads);
     }
-    if (t == 0 && lse_ptr) *lse_ptr = M == kNegInf ? kNegInf : (M + log2f(L)) * kLn2;
+    if (t == 0 && lse_ptr) *lse_ptr = M == kNegInf ? kNegInf : (M + log2f(Lx)) * kLn2;
 }
 
 }  // namespace dev

@@ -1,0 +1,764 @@
+// td_gqa -- grouped-query / multi-query split-KV decode on the sm_100a
+// tensor cores (tcgen05 + TMEM).
+//
+// What it computes: as td_partial ("Tree Attention Decoding" gist, Algorithm
+// 3), but G = Hq / Hkv query heads share each key/value head, so one pass over
+// a K/V tile serves G queries.  The tile work is then a small dense
+// contraction: S = Q K^T with Q [G x D] and P V with P [G x keys], which this
+// kernel issues to the 5th-generation tensor cores with the query heads on
+// the MMA's M axis (M = 128, rows >= G are zero).
+//
+// The keys of all (b, kv-head) sequences form one flattened space split evenly
+// over the CTAs, exactly as in td_partial; pieces of a sequence cut across CTAs
+// are merged by the last CTA to finish (atomic ticket), per query head.
+//
+// One CTA per SM, 6 warps:
+//   warp 0      TMA producer: K and V tiles of 64 keys, 2-D tensor-map loads
+//               with 128-byte swizzle (one box per 64 columns of D), 4 stages;
+//   warp 1      allocates 256 TMEM columns and issues the MMAs from one lane:
+//               S(t) = Q K(t)^T into one of two S buffers, then O += P(t) V(t)
+//               into the O accumulator, completion signalled by tcgen05.commit;
+//   warps 2-5   softmax warpgroup (warp w reads TMEM lanes 32*(w%4)..+31, one
+//               query head per lane): read S, scale, ALiBi term, row max,
+//               p = 2^(s - m) rounded to the input type and written to shared
+//               memory as the A operand of the P V product; at the end of a
+//               piece read O and write the output or a part record.
+// The running max m of a row is only moved when a tile's max exceeds it by
+// more than 8 (log2 units); O in TMEM is rescaled then, and p <= 2^8 otherwise.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <type_traits>
+
+#include "td_device.cuh"
+#include "td_internal.cuh"
+#include "treedec.h"
+
+namespace td {
+namespace {
+
+using namespace dev;
+
+constexpr int kTK = 64;            // keys per tile
+constexpr int kM = 128;            // MMA rows (query heads, padded)
+constexpr int kGqaStages = 4;      // K/V pipeline depth
+constexpr int kGqaThreads = 192;   // 6 warps
+constexpr int kSoftmaxThreads = 128;
+constexpr int kTmemCols = 256;     // S0 [0,64) S1 [64,128) O [128,128+D)
+constexpr int kScratchFloats = 1024;
+constexpr float kRescaleThreshold = 8.f;  // log2 units
+
+template <int D>
+struct GCfg {
+    static constexpr int kAtoms = D / 64;                    // 64-column swizzle atoms
+    static constexpr int kQBytes = kAtoms * kM * 128;        // Q, K-major SW128
+    static constexpr int kPBytes = kM * 128;                 // one P buffer (64 keys)
+    static constexpr int kKVAtomBytes = kTK * 128;           // 64 keys x 64 columns
+    static constexpr int kStageBytes = 2 * kAtoms * kKVAtomBytes;  // K atoms, then V atoms
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffP = kOffQ + kQBytes;
+    static constexpr int kOffKV = kOffP + 2 * kPBytes;
+    static constexpr int kOffScratch = kOffKV + kGqaStages * kStageBytes;
+    static constexpr size_t kSmem = size_t(kOffScratch) + kScratchFloats * 4 + 1024;  // +align
+    static_assert(D == 64 || D == 128, "D");
+};
+
+struct GCtl {
+    long long T, x0, x1, b0, pre0;
+    int abort;
+    int last;
+    uint32_t tmem;
+};
+
+// ------------------------------------------------------------ tcgen05 PTX
+
+__device__ __forceinline__ void fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16, one CTA
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                         uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// arrive on `bar` when every tcgen05 op issued so far by this thread is done
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+          "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+          "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+          "=r"(r[31])
+        : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+          "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+          "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+          "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+          "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// 2-D tiled TMA load (no multicast) of box {64 columns, 64 rows}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(pol)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle, sm_100 format (version 1).
+// lbo/sbo in bytes.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= uint64_t((addr >> 4) & 0x3FFFu);
+    d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+    d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
+    d |= uint64_t(1) << 46;  // descriptor version for sm_100
+    d |= uint64_t(2) << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16, fp32 accumulate.  ab: 0 = f16, 1 = bf16.
+__host__ __device__ constexpr uint32_t instr_desc_f16(int ab, int m, int n, int a_mn, int b_mn) {
+    return (1u << 4) | (uint32_t(ab) << 7) | (uint32_t(ab) << 10) | (uint32_t(a_mn) << 15) |
+           (uint32_t(b_mn) << 16) | (uint32_t(n >> 3) << 17) | (uint32_t(m >> 4) << 24);
+}
+
+// offset of 16-byte chunk c of row r inside a 128-byte-swizzled block
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+    return uint32_t(r) * 128u + (uint32_t(c ^ (r & 7)) << 4);
+}
+
+__device__ __forceinline__ uint32_t pack_round(float a, float b, bool bf16, float& ra, float& rb) {
+    uint32_t w;
+    if (bf16) {
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(b), "f"(a));
+        ra = __uint_as_float(w << 16);
+        rb = __uint_as_float(w & 0xffff0000u);
+    } else {
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(b), "f"(a));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+        ra = f.x;
+        rb = f.y;
+    }
+    return w;
+}
+
+// ------------------------------------------------------------- the kernel
+
+// Part record of one query head: num[D], m (log2 units), l of the rounded p
+// (normalises num), l of the unrounded p (for lse).
+struct GSlotAcc {
+    static constexpr bool kSplitL = true;
+    const float* part;
+    long long c_lo;
+    int first_slot, G, g, D;
+    __device__ __forceinline__ const float* rec(int i) const {
+        const long long c = c_lo + i;
+        const int slot = i == 0 ? first_slot : 0;
+        return part + ((c * 2 + slot) * G + g) * (D + 3);
+    }
+    __device__ __forceinline__ float m2(int i) const { return __ldcg(rec(i) + D); }
+    __device__ __forceinline__ float l(int i) const { return __ldcg(rec(i) + D + 1); }
+    __device__ __forceinline__ float lx(int i) const { return __ldcg(rec(i) + D + 2); }
+    __device__ __forceinline__ float num(int i, int d) const { return __ldcg(rec(i) + d); }
+};
+
+__device__ __forceinline__ long long gseq_len(const GqaParams& p, int b) {
+    int n = __ldg(p.seqlens + b);
+    if (n < 0 || n > p.N) {
+        atomicOr(p.err, TD_DEVERR_BAD_SEQLEN);
+        n = n < 0 ? 0 : static_cast<int>(p.N);
+    }
+    return n;
+}
+
+struct GWalk {
+    long long start, len, pre;
+    int b, h;  // h: kv head
+};
+
+__device__ __forceinline__ bool gwalk_first(const GqaParams& p, const GCtl& ctl, GWalk& w) {
+    if (ctl.x0 >= ctl.x1) return false;
+    if (p.seqlens == nullptr) {
+        const long long g = ctl.x0 / p.N;
+        w.b = static_cast<int>(g / p.Hkv);
+        w.h = static_cast<int>(g % p.Hkv);
+        w.start = g * p.N;
+        w.len = p.N;
+        w.pre = 0;
+    } else {
+        w.b = static_cast<int>(ctl.b0);
+        w.pre = ctl.pre0;
+        w.len = gseq_len(p, w.b);
+        w.h = static_cast<int>((ctl.x0 - p.Hkv * w.pre) / w.len);
+        w.start = p.Hkv * w.pre + w.h * w.len;
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool gwalk_next(const GqaParams& p, const GCtl& ctl, GWalk& w) {
+    if (p.seqlens == nullptr) {
+        if (++w.h == p.Hkv) {
+            w.h = 0;
+            ++w.b;
+        }
+        w.start += p.N;
+    } else {
+        if (++w.h == p.Hkv) {
+            w.h = 0;
+            w.pre += w.len;
+            do {
+                ++w.b;
+            } while (w.b < p.B && (w.len = gseq_len(p, w.b)) == 0);
+            if (w.b >= p.B) return false;
+        }
+        w.start = p.Hkv * w.pre + w.h * w.len;
+    }
+    return w.start < ctl.x1;
+}
+
+__device__ __forceinline__ long long gpart_start(long long c, long long T, long long P) {
+    return c * T / P;
+}
+__device__ __forceinline__ long long gpart_of(long long x, long long T, long long P) {
+    return ((x + 1) * P - 1) / T;
+}
+
+constexpr int kBarSoftmax = 1;
+
+template <typename E, int D>
+__global__ void __launch_bounds__(kGqaThreads, 1)
+    td_gqa_kernel(const GqaParams p, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV) {
+    using C = GCfg<D>;
+    constexpr bool kBF16 = std::is_same<E, __nv_bfloat16>::value;
+    extern __shared__ unsigned char smem_raw[];
+    // 1024-byte alignment for the swizzled operand blocks
+    unsigned char* smem = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* scratch = reinterpret_cast<float*>(smem + C::kOffScratch);
+
+    __shared__ __align__(8) uint64_t kv_full[kGqaStages], kv_empty[kGqaStages];
+    __shared__ __align__(8) uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2], q_ready;
+    __shared__ GCtl ctl;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const long long c = blockIdx.x;
+    const long long P = p.P;
+    const int G = p.G;
+
+    if (tid == 0) {
+        for (int s = 0; s < kGqaStages; ++s) {
+            mbar_init(smem_addr(&kv_full[s]), 1);
+            mbar_init(smem_addr(&kv_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&s_full[s]), 1);
+            mbar_init(smem_addr(&s_empty[s]), 4);
+            mbar_init(smem_addr(&p_full[s]), 4);
+            mbar_init(smem_addr(&pv_done[s]), 1);
+        }
+        mbar_init(smem_addr(&q_ready), 4);
+        fence_barrier_init();
+        ctl.abort = 0;
+        ctl.last = 0;
+    }
+    if (warp == 1) {
+        // TMEM: 256 columns, address written to ctl.tmem
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_addr(&ctl.tmem)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp >= 2) {
+        // Q and both P buffers start at zero (rows >= G stay zero)
+        uint4* z = reinterpret_cast<uint4*>(smem + C::kOffQ);
+        const int n16 = (C::kQBytes + 2 * C::kPBytes) / 16;
+        for (int i = tid - 64; i < n16; i += kSoftmaxThreads) z[i] = make_uint4(0, 0, 0, 0);
+        fence_proxy_async_smem();
+    }
+    if (p.seqlens == nullptr) {
+        if (tid == 0) {
+            ctl.T = p.T;
+            ctl.x0 = gpart_start(c, p.T, P);
+            ctl.x1 = gpart_start(c + 1, p.T, P);
+            ctl.b0 = 0;
+            ctl.pre0 = 0;
+        }
+    } else {
+        if (warp == 0) {
+            long long sum = 0;
+            for (int b = lane; b < p.B; b += 32) sum += gseq_len(p, b);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+            const long long T = sum * p.Hkv;
+            const long long x0 = T > 0 ? gpart_start(c, T, P) : 0;
+            const long long x1 = T > 0 ? gpart_start(c + 1, T, P) : 0;
+            long long b0 = p.B, pre0 = sum;
+            if (x0 < x1) {
+                long long run = 0;
+                for (int base = 0; base < p.B; base += 32) {
+                    const int b = base + lane;
+                    const long long n = b < p.B ? gseq_len(p, b) : 0;
+                    long long incl = n;
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const long long y = __shfl_up_sync(0xffffffffu, incl, o);
+                        if (lane >= o) incl += y;
+                    }
+                    const bool hit = b < p.B && p.Hkv * (run + incl) > x0;
+                    const unsigned m = __ballot_sync(0xffffffffu, hit);
+                    if (m) {
+                        const int L = __ffs(m) - 1;
+                        const long long inclL = __shfl_sync(0xffffffffu, incl, L);
+                        const long long nL = __shfl_sync(0xffffffffu, n, L);
+                        b0 = base + L;
+                        pre0 = run + inclL - nL;
+                        break;
+                    }
+                    run += __shfl_sync(0xffffffffu, incl, 31);
+                }
+            }
+            if (lane == 0) {
+                ctl.T = T;
+                ctl.x0 = x0;
+                ctl.x1 = x1;
+                ctl.b0 = b0;
+                ctl.pre0 = pre0;
+            }
+        }
+        for (long long b = c; b < p.B; b += P) {
+            if (gseq_len(p, static_cast<int>(b)) != 0) continue;
+            for (int i = tid; i < p.Hq * D; i += kGqaThreads) p.out[b * p.Hq * D + i] = 0.f;
+            if (p.lse)
+                for (int h = tid; h < p.Hq; h += kGqaThreads) p.lse[b * p.Hq + h] = kNegInf;
+        }
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+
+    const long long T = ctl.T, x0 = ctl.x0, x1 = ctl.x1;
+    const uint32_t tmem = ctl.tmem;
+    volatile int* abort_flag = &ctl.abort;
+    const uint32_t sQ = smem_addr(smem + C::kOffQ);
+    const uint32_t sP = smem_addr(smem + C::kOffP);
+    const uint32_t sKV = smem_addr(smem + C::kOffKV);
+
+    if (warp == 0) {
+        // -------------------------------------------------------- producer
+        if (lane == 0) {
+            const uint64_t pol = l2_policy_evict_first();
+            int stage = 0;
+            uint32_t phase = 0;
+            long long issued = 0;
+            bool aborted = false;
+            GWalk w;
+            if (gwalk_first(p, ctl, w)) {
+                do {
+                    const long long j0 = (x0 > w.start ? x0 : w.start) - w.start;
+                    const long long e = w.start + w.len;
+                    const long long j1 = (x1 < e ? x1 : e) - w.start;
+                    const long long rowbase = (static_cast<long long>(w.b) * p.Hkv + w.h) * p.N;
+                    for (long long t0 = j0; t0 < j1; t0 += kTK) {
+                        if (!aborted &&
+                            !mbar_wait_bounded(smem_addr(&kv_empty[stage]), phase ^ 1u, abort_flag,
+                                               p.err, TD_DEVERR_WAIT_TIMEOUT))
+                            aborted = true;
+                        if (!aborted) {
+                            const uint32_t fb = smem_addr(&kv_full[stage]);
+                            const uint32_t base = sKV + stage * C::kStageBytes;
+                            const int y = static_cast<int>(rowbase + t0);
+                            mbar_arrive_expect_tx(fb, C::kStageBytes);
+#pragma unroll
+                            for (int a = 0; a < C::kAtoms; ++a) {
+                                tma_load_2d(base + a * C::kKVAtomBytes, &tmK, 64 * a, y, fb, pol);
+                                tma_load_2d(base + (C::kAtoms + a) * C::kKVAtomBytes, &tmV, 64 * a,
+                                            y, fb, pol);
+                            }
+                            ++issued;
+                        }
+                        if (++stage == kGqaStages) {
+                            stage = 0;
+                            phase ^= 1u;
+                        }
+                    }
+                } while (gwalk_next(p, ctl, w));
+            }
+            for (int s = 0; s < kGqaStages && s < issued; ++s) {
+                const long long lastTile = s + ((issued - 1 - s) / kGqaStages) * kGqaStages;
+                mbar_wait_bounded(smem_addr(&kv_full[s]),
+                                  static_cast<uint32_t>((lastTile / kGqaStages) & 1), nullptr,
+                                  p.err, TD_DEVERR_WAIT_TIMEOUT);
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA
+        if (lane == 0) {
+            constexpr uint32_t idS = instr_desc_f16(kBF16 ? 1 : 0, kM, kTK, 0, 0);
+            constexpr uint32_t idO = instr_desc_f16(kBF16 ? 1 : 0, kM, D, 0, 1);
+            long long t = 0;    // tiles issued so far (global)
+            long long pc = 0;   // pieces so far
+            bool aborted = false;
+            long long last_pv = -1;
+            auto wait = [&](uint64_t* bar, uint32_t par) {
+                if (!aborted && !mbar_wait_bounded(smem_addr(bar), par, abort_flag, p.err,
+                                                   TD_DEVERR_WAIT_TIMEOUT))
+                    aborted = true;
+            };
+            auto issue_S = [&](long long tt) {
+                const int stage = static_cast<int>(tt % kGqaStages);
+                wait(&kv_full[stage], static_cast<uint32_t>((tt / kGqaStages) & 1));
+                if (tt >= 2) wait(&s_empty[tt & 1], static_cast<uint32_t>(((tt >> 1) - 1) & 1));
+                fence_after();
+                const uint32_t kb = sKV + stage * C::kStageBytes;
+                const uint32_t dS = tmem + static_cast<uint32_t>((tt & 1) * kTK);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);  // 16 cols in the atom
+                    const uint64_t a = smem_desc_sw128(sQ + (kk >> 2) * (kM * 128) + off, 16, 1024);
+                    const uint64_t b = smem_desc_sw128(kb + (kk >> 2) * C::kKVAtomBytes + off, 16, 1024);
+                    umma_f16(dS, a, b, idS, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(smem_addr(&s_full[tt & 1]));
+            };
+            GWalk w;
+            if (gwalk_first(p, ctl, w)) {
+                do {
+                    const long long j0 = (x0 > w.start ? x0 : w.start) - w.start;
+                    const long long e = w.start + w.len;
+                    const long long j1 = (x1 < e ? x1 : e) - w.start;
+                    const long long nt = (j1 - j0 + kTK - 1) / kTK;
+                    wait(&q_ready, static_cast<uint32_t>(pc & 1));
+                    fence_after();
+                    issue_S(t);
+                    for (long long i = 0; i < nt; ++i, ++t) {
+                        if (i + 1 < nt) issue_S(t + 1);
+                        wait(&p_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+                        fence_after();
+                        const int stage = static_cast<int>(t % kGqaStages);
+                        const uint32_t vb = sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtomBytes;
+                        const uint32_t pb = sP + static_cast<uint32_t>((t & 1) * C::kPBytes);
+#pragma unroll
+                        for (int kk = 0; kk < kTK / 16; ++kk) {
+                            const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
+                            const uint64_t b =
+                                smem_desc_sw128(vb + kk * 2048, C::kKVAtomBytes, 1024);
+                            umma_f16(tmem + 128, a, b, idO, (i > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        umma_commit(smem_addr(&pv_done[t & 1]));
+                        umma_commit(smem_addr(&kv_empty[stage]));
+                        last_pv = t;
+                    }
+                    ++pc;
+                } while (gwalk_next(p, ctl, w));
+            }
+            // every MMA must be complete before the CTA frees TMEM
+            if (last_pv >= 0)
+                mbar_wait_bounded(smem_addr(&pv_done[last_pv & 1]),
+                                  static_cast<uint32_t>((last_pv >> 1) & 1), nullptr, p.err,
+                                  TD_DEVERR_WAIT_TIMEOUT);
+        }
+        __syncwarp();
+    } else {
+        // --------------------------------------------------------- softmax
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;      // MMA row = query head within the group
+        const bool warp_active = quarter * 32 < G;
+        const bool active = r < G;
+        const int st = tid - 64;                // 0..127 within the softmax warpgroup
+        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+        const float qscale2 = p.qscale2;
+        long long t = 0;
+        long long pc = 0;
+        bool aborted = false;
+        auto wait = [&](uint64_t* bar, uint32_t par) {
+            if (!aborted && !mbar_wait_bounded(smem_addr(bar), par, abort_flag, p.err,
+                                               TD_DEVERR_WAIT_TIMEOUT))
+                aborted = true;
+        };
+        GWalk w;
+        if (gwalk_first(p, ctl, w)) {
+            do {
+                const long long j0 = (x0 > w.start ? x0 : w.start) - w.start;
+                const long long e = w.start + w.len;
+                const long long j1 = (x1 < e ? x1 : e) - w.start;
+                const long long nt = (j1 - j0 + kTK - 1) / kTK;
+                const bool whole = (j0 == 0 && j1 == w.len);
+                const long long hq = static_cast<long long>(w.h) * G + r;          // query head
+                const long long qrow = static_cast<long long>(w.b) * p.Hq + hq;   // b*Hq + hq
+                // Q rows of this kv head's group, K-major, 128-byte swizzle
+                if (active) {
+                    const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) + qrow * D);
+#pragma unroll
+                    for (int a = 0; a < C::kAtoms; ++a)
+#pragma unroll
+                        for (int cc = 0; cc < 8; ++cc) {
+                            const uint4 v = __ldg(qg + a * 8 + cc);
+                            *reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kM * 128) + swz(r, cc)) = v;
+                        }
+                }
+                fence_proxy_async_smem();
+                fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&q_ready));
+
+                const float slope2 =
+                    (active && p.slopes) ? __ldg(p.slopes + hq) * kLog2e : 0.f;
+                // l: sum of p as rounded for the P V product (normalises O);
+                // lx: sum of the unrounded p (for lse)
+                float m_ref = kNegInf, l = 0.f, lx = 0.f;
+                for (long long i = 0; i < nt; ++i, ++t) {
+                    const long long t0 = j0 + i * kTK;
+                    const int rows = static_cast<int>((j1 - t0) < kTK ? (j1 - t0) : kTK);
+                    wait(&s_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+                    fence_after();
+                    uint32_t sr[2][32];
+                    if (warp_active) {
+                        const uint32_t sa = tmem + lane_addr + static_cast<uint32_t>((t & 1) * kTK);
+                        tmem_ld32(sa, sr[0]);
+                        tmem_ld32(sa + 32, sr[1]);
+                        tmem_wait_ld();
+                    }
+                    fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&s_empty[t & 1]));
+
+                    if (rows < kTK) {
+                        // keys past the piece end: the tile holds other rows (or padding
+                        // that may not be finite); p is 0 there, and 0 * NaN would poison
+                        // O, so zero those V rows before the P V product reads them
+                        const int stage = static_cast<int>(t % kGqaStages);
+                        unsigned char* vb = smem + C::kOffKV + stage * C::kStageBytes +
+                                            C::kAtoms * C::kKVAtomBytes;
+                        const int n16 = (kTK - rows) * 8 * C::kAtoms;  // 16-B units to clear
+                        for (int i = lane + quarter * 32; i < n16; i += kSoftmaxThreads) {
+                            const int a = i / ((kTK - rows) * 8);
+                            const int rem = i - a * ((kTK - rows) * 8);
+                            const int row = rows + rem / 8, cc = rem % 8;
+                            *reinterpret_cast<uint4*>(vb + a * C::kKVAtomBytes + swz(row, cc)) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    if (warp_active) {
+                        float s[kTK];
+                        float mt = kNegInf;
+#pragma unroll
+                        for (int k = 0; k < kTK; ++k) {
+                            const float raw = __uint_as_float(sr[k >> 5][k & 31]);
+                            float v = p.slopes ? fmaf(raw, qscale2,
+                                                      slope2 * static_cast<float>(t0 + k - w.len + 1))
+                                               : raw * qscale2;
+                            v = (k < rows && active) ? v : kNegInf;
+                            s[k] = v;
+                            mt = fmaxf(mt, v);
+                        }
+                        const bool need = active && (m_ref == kNegInf ? mt != kNegInf
+                                                                       : mt > m_ref + kRescaleThreshold);
+                        const float m_new = need ? fmaxf(m_ref, mt) : m_ref;
+                        const float factor = need ? rescale(m_ref, m_new) : 1.f;
+                        if (__any_sync(0xffffffffu, need && i > 0)) {
+                            // O already holds earlier tiles of this piece: scale it
+                            wait(&pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+                            fence_after();
+#pragma unroll 1
+                            for (int cc = 0; cc < D / 32; ++cc) {
+                                uint32_t o[32];
+                                const uint32_t oa = tmem + lane_addr + 128 + cc * 32;
+                                tmem_ld32(oa, o);
+                                tmem_wait_ld();
+#pragma unroll
+                                for (int x = 0; x < 32; ++x)
+                                    o[x] = __float_as_uint(__uint_as_float(o[x]) * factor);
+                                tmem_st32(oa, o);
+                            }
+                            tmem_wait_st();
+                        }
+                        l *= factor;
+                        lx *= factor;
+                        m_ref = m_new;
+                        // P buffer (t & 1) was read by the P V product of tile t - 2
+                        if (t >= 2)
+                            wait(&pv_done[t & 1], static_cast<uint32_t>(((t >> 1) - 1) & 1));
+                        if (active) {
+                            unsigned char* prow = smem + C::kOffP + (t & 1) * C::kPBytes;
+#pragma unroll
+                            for (int cc = 0; cc < 8; ++cc) {
+                                float e[8];
+                                uint32_t w4[4];
+                                float lsum = 0.f, xsum = 0.f;
+#pragma unroll
+                                for (int x = 0; x < 8; ++x) {
+                                    e[x] = ex2(s[cc * 8 + x] - m_ref);
+                                    xsum += e[x];
+                                }
+#pragma unroll
+                                for (int x = 0; x < 4; ++x) {
+                                    float ra, rb;
+                                    w4[x] = pack_round(e[2 * x], e[2 * x + 1], kBF16, ra, rb);
+                                    lsum += ra + rb;
+                                }
+                                l += lsum;
+                                lx += xsum;
+                                *reinterpret_cast<uint4*>(prow + swz(r, cc)) =
+                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                            }
+                        }
+                        fence_proxy_async_smem();
+                    }
+                    fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&p_full[t & 1]));
+                }
+
+                // ---- end of piece: O rows of this group
+                float* rec = nullptr;
+                const int slot = pc == 0 ? 0 : 1;  // first piece of the CTA uses slot 0
+                if (warp_active) {
+                    wait(&pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+                    fence_after();
+                    if (!whole) rec = p.part + ((c * 2 + slot) * G + r) * (D + 3);
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        tmem_ld32(tmem + lane_addr + 128 + cc * 32, o);
+                        tmem_wait_ld();
+                        if (active) {
+                            if (whole) {
+                                float* dst = p.out + qrow * D + cc * 32;
+#pragma unroll
+                                for (int x = 0; x < 32; ++x) dst[x] = __uint_as_float(o[x]) / l;
+                            } else {
+#pragma unroll
+                                for (int x = 0; x < 32; ++x) rec[cc * 32 + x] = __uint_as_float(o[x]);
+                            }
+                        }
+                    }
+                    if (active) {
+                        if (whole) {
+                            if (p.lse) p.lse[qrow] = (m_ref + log2f(lx)) * kLn2;
+                        } else {
+                            rec[D] = m_ref;
+                            rec[D + 1] = l;
+                            rec[D + 2] = lx;
+                        }
+                    }
+                    fence_before();
+                }
+                if (!whole) {
+                    __threadfence();
+                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                    const long long c_lo = gpart_of(w.start, T, P);
+                    const long long c_hi = gpart_of(w.start + w.len - 1, T, P);
+                    const int n = static_cast<int>(c_hi - c_lo + 1);
+                    const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+                    if (st == 0) {
+                        const int prev = atomicAdd(p.tickets + seg, 1);
+                        const int last = prev == n - 1;
+                        if (last) atomicExch(p.tickets + seg, 0);
+                        ctl.last = last;
+                    }
+                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                    if (ctl.last) {
+                        __threadfence();
+                        const int first_slot = gpart_start(c_lo, T, P) < w.start ? 1 : 0;
+                        for (int g = 0; g < G; ++g) {
+                            const long long orow = static_cast<long long>(w.b) * p.Hq +
+                                                   static_cast<long long>(w.h) * G + g;
+                            const GSlotAcc acc{p.part, c_lo, first_slot, G, g, D};
+                            tree_merge(acc, n, D, st, kSoftmaxThreads, scratch, kScratchFloats,
+                                       kBarSoftmax, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+                        }
+                    }
+                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                }
+                ++pc;
+            } while (gwalk_next(p, ctl, w));
+        }
+    }
+
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(kTmemCols) : "memory");
+    }
+}
+
+template <typename E, int D>
+cudaError_t launch_gqa_t(int device, const GqaParams& p, const CUtensorMap& mk,
+                         const CUtensorMap& mv, cudaStream_t s) {
+    using C = GCfg<D>;
+    auto kern = td_gqa_kernel<E, D>;
+    static std::atomic<unsigned long long> configured{0};
+    const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
+    if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(C::kSmem));
+        if (e != cudaSuccess) return e;
+        configured.fetch_or(bit, std::memory_order_acq_rel);
+    }
+    kern<<<static_cast<unsigned>(p.P), kGqaThreads, C::kSmem, s>>>(p, mk, mv);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t gqa_smem_bytes(int D) {
+    return D == 64 ? GCfg<64>::kSmem : D == 128 ? GCfg<128>::kSmem : 0;
+}
+
+cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const CUtensorMap& mk,
+                       const CUtensorMap& mv, cudaStream_t s) {
+    if (dtype == kBF16) {
+        if (D == 64) return launch_gqa_t<__nv_bfloat16, 64>(device, p, mk, mv, s);
+        if (D == 128) return launch_gqa_t<__nv_bfloat16, 128>(device, p, mk, mv, s);
+    } else if (dtype == kF16) {
+        if (D == 64) return launch_gqa_t<__half, 64>(device, p, mk, mv, s);
+        if (D == 128) return launch_gqa_t<__half, 128>(device, p, mk, mv, s);
+    }
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace td

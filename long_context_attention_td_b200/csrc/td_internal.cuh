@@ -2,6 +2,7 @@
 // libtreedec.  Not part of the C ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -59,6 +60,27 @@ struct PartialParams {
     int* tickets;            // [B*H]
     int* err;                // error word
 };
+
+// Grouped-query kernel (td_gqa.cu): Hq = G * Hkv query heads over Hkv kv heads.
+struct GqaParams {
+    const void* q;           // [B, Hq, 1, D]
+    float* out;              // [B, Hq, 1, D]
+    float* lse;              // [B, Hq, 1] or null
+    const float* slopes;     // [Hq] or null
+    const int32_t* seqlens;  // [B] or null
+    int B, Hq, Hkv, G;
+    int64_t N;               // keys per sequence, or the padded Nmax
+    int64_t T;               // attended keys over all (b, kv head) when uniform, else -1
+    int64_t P;               // parts == grid size
+    float qscale2;           // D^-1/2 * log2(e)
+    float* part;             // part records [P][2][G][D + 3]
+    int* tickets;            // [B * Hkv]
+    int* err;
+};
+size_t gqa_smem_bytes(int D);
+// K and V tensor maps: 2-D [B*Hkv*N rows, D columns], box {64, 64}, 128-byte swizzle.
+cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const CUtensorMap& mk,
+                       const CUtensorMap& mv, cudaStream_t s);
 
 // Dynamic shared memory of the split-KV kernel for (dtype, D).
 size_t partial_smem_bytes(int dtype, int D);

@@ -128,6 +128,7 @@ __device__ __forceinline__ bool walk_next(const PartialParams& p, const Ctl& ctl
 
 // Part records written by the CTAs that share one sequence, for tree_merge.
 struct SlotAcc {
+    static constexpr bool kSplitL = false;
     const float* part;
     long long c_lo;
     int first_slot;

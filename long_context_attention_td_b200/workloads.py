@@ -100,6 +100,24 @@ def _randn_rows(gen, rows, D, device, scale, dtype):
     return out
 
 
+def make_gqa_inputs(w: Workload, Hkv: int, device="cpu"):
+    """Grouped-query inputs: q [B, w.H, 1, D], k/v [B, Hkv, N, D] (same recipe
+    as make_inputs, with the key/value tensors drawn for Hkv heads)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    B, H, D, N = w.B, w.H, w.D, w.N
+    qf = torch.randn((B, H, 1, D), generator=g, device=device, dtype=torch.float32)
+    if w.scale != 1.0:
+        qf.mul_(w.scale)
+    q = qf.to(w.dtype)
+    k = _randn_rows(g, B * Hkv * N, D, device, w.scale, w.dtype).view(B, Hkv, N, D)
+    v = _randn_rows(g, B * Hkv * N, D, device, w.scale, w.dtype).view(B, Hkv, N, D)
+    sl_host = seqlens_for(w)
+    slopes = alibi_slopes(H, device) if w.alibi else None
+    seqlens = sl_host.to(device) if sl_host is not None else None
+    return dict(q=q, k=k, v=v, slopes=slopes, seqlens=seqlens, seqlens_host=sl_host)
+
+
 def make_inputs(w: Workload, device="cpu"):
     """Materialise a workload: dict(q, k, v, slopes, seqlens, seqlens_host)."""
     device = torch.device(device)
