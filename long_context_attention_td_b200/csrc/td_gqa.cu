@@ -60,7 +60,10 @@ struct GCfg {
     static constexpr int kOffP = kOffQ + kQBytes;
     static constexpr int kOffKV = kOffP + 2 * kPBytes;
     static constexpr int kOffScratch = kOffKV + kGqaStages * kStageBytes;
-    static constexpr size_t kSmem = size_t(kOffScratch) + kScratchFloats * 4 + 1024;  // +align
+    // end-of-piece staging of the replicas' O rows: 128 rows x 32 columns, row stride 33
+    static constexpr int kOffStage = kOffScratch + kScratchFloats * 4;
+    static constexpr int kStageFloats = kM * 33;
+    static constexpr size_t kSmem = size_t(kOffStage) + kStageFloats * 4 + 1024;  // +align
     static_assert(D == 64 || D == 128, "D");
 };
 
@@ -265,7 +268,313 @@ __device__ __forceinline__ long long gpart_of(long long x, long long T, long lon
 
 constexpr int kBarSoftmax = 1;
 
-template <typename E, int D>
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+struct SmCtx {
+    unsigned char* smem;
+    float* scratch;
+    uint64_t* s_full;
+    uint64_t* s_empty;
+    uint64_t* p_full;
+    uint64_t* pv_done;
+    uint64_t* q_ready;
+    GCtl* ctl;
+    volatile int* abort_flag;
+    uint32_t tmem;
+    long long T, x0, x1, P, c;
+    int warp, lane, tid;
+};
+
+// The softmax warpgroup.  The G query rows are replicated R = 64 / CW times
+// across the TMEM lane quarters (rows rep*RR + g, RR = 128 / R); replica rep
+// handles key columns [rep*CW, rep*CW + CW) of every tile as an independent
+// split with its own running max, so all four warps share the exponentials.
+// At the end of a piece the replicas are merged in shared memory.
+template <typename E, int D, int CW>
+__device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x) {
+    using C = GCfg<D>;
+    constexpr bool kBF16 = std::is_same<E, __nv_bfloat16>::value;
+    constexpr int R = kTK / CW;   // replicas
+    constexpr int RR = kM / R;    // MMA rows per replica
+    const int G = p.G;
+    const int quarter = x.warp & 3;
+    const int r = quarter * 32 + x.lane;  // MMA row (TMEM lane)
+    const int rep = r / RR;               // replica: key-column slice of each tile
+    const int g = r - rep * RR;           // query head within the group
+    const bool warp_active = ((quarter * 32) % RR) < G;
+    const bool active = g < G;
+    const int st = x.tid - 64;            // 0..127 within the warpgroup
+    const int lane = x.lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const int cb = rep * CW;              // first key column of this replica
+    const float qscale2 = p.qscale2;
+    unsigned char* smem = x.smem;
+    float* stage = reinterpret_cast<float*>(smem + C::kOffStage);
+    long long t = 0;
+    long long pc = 0;
+    bool aborted = false;
+    auto wait = [&](uint64_t* bar, uint32_t par) {
+        if (!aborted && !mbar_wait_bounded(smem_addr(bar), par, x.abort_flag, p.err,
+                                           TD_DEVERR_WAIT_TIMEOUT))
+            aborted = true;
+    };
+    GWalk w;
+    if (!gwalk_first(p, *x.ctl, w)) return;
+    do {
+        const long long j0 = (x.x0 > w.start ? x.x0 : w.start) - w.start;
+        const long long e = w.start + w.len;
+        const long long j1 = (x.x1 < e ? x.x1 : e) - w.start;
+        const long long nt = (j1 - j0 + kTK - 1) / kTK;
+        const bool whole = (j0 == 0 && j1 == w.len);
+        const long long hq = static_cast<long long>(w.h) * G + g;          // query head
+        const long long qrow = static_cast<long long>(w.b) * p.Hq + hq;   // b*Hq + hq
+        // Q rows of this kv head's group (each replica a copy), K-major SW128
+        if (active) {
+            const uint4* qg =
+                reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) + qrow * D);
+#pragma unroll
+            for (int a = 0; a < C::kAtoms; ++a)
+#pragma unroll
+                for (int cc = 0; cc < 8; ++cc)
+                    *reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kM * 128) + swz(r, cc)) =
+                        __ldg(qg + a * 8 + cc);
+        }
+        fence_proxy_async_smem();
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(x.q_ready));
+
+        const float slope2 = (active && p.slopes) ? __ldg(p.slopes + hq) * kLog2e : 0.f;
+        // l: sum of p as rounded for the P V product (normalises O);
+        // lx: sum of the unrounded p (for lse)
+        float m_ref = kNegInf, l = 0.f, lx = 0.f;
+        for (long long i = 0; i < nt; ++i, ++t) {
+            const long long t0 = j0 + i * kTK;
+            const int rows = static_cast<int>((j1 - t0) < kTK ? (j1 - t0) : kTK);
+            wait(&x.s_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+            fence_after();
+            uint32_t sr[CW];
+            if (warp_active) {
+                const uint32_t sa =
+                    x.tmem + lane_addr + static_cast<uint32_t>((t & 1) * kTK + cb);
+                if constexpr (CW == 16) {
+                    tmem_ld16(sa, sr);
+                } else {
+#pragma unroll
+                    for (int h = 0; h < CW / 32; ++h)
+                        tmem_ld32(sa + 32 * h, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * h));
+                }
+                tmem_wait_ld();
+            }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[t & 1]));
+
+            if (rows < kTK) {
+                // keys past the piece end: the tile holds other rows (or padding
+                // that may not be finite); p is 0 there, and 0 * NaN would poison
+                // O, so zero those V rows before the P V product reads them
+                const int stg = static_cast<int>(t % kGqaStages);
+                unsigned char* vb =
+                    smem + C::kOffKV + stg * C::kStageBytes + C::kAtoms * C::kKVAtomBytes;
+                const int per_atom = (kTK - rows) * 8;  // 16-B units per atom
+                for (int u = st; u < per_atom * C::kAtoms; u += kSoftmaxThreads) {
+                    const int a = u / per_atom;
+                    const int rem = u - a * per_atom;
+                    *reinterpret_cast<uint4*>(vb + a * C::kKVAtomBytes +
+                                              swz(rows + rem / 8, rem % 8)) = make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async_smem();
+            }
+            if (warp_active) {
+                float sv[CW];
+                float mt = kNegInf;
+#pragma unroll
+                for (int k = 0; k < CW; ++k) {
+                    const int col = cb + k;
+                    const float raw = __uint_as_float(sr[k]);
+                    float v = p.slopes
+                                  ? fmaf(raw, qscale2, slope2 * static_cast<float>(t0 + col - w.len + 1))
+                                  : raw * qscale2;
+                    v = (col < rows && active) ? v : kNegInf;
+                    sv[k] = v;
+                    mt = fmaxf(mt, v);
+                }
+                const bool need = active && (m_ref == kNegInf ? mt != kNegInf
+                                                               : mt > m_ref + kRescaleThreshold);
+                const float m_new = need ? fmaxf(m_ref, mt) : m_ref;
+                const float factor = need ? rescale(m_ref, m_new) : 1.f;
+                if (__any_sync(0xffffffffu, need && m_ref != kNegInf)) {
+                    // O already holds earlier tiles of this piece: scale it
+                    wait(&x.pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+                    fence_after();
+#pragma unroll 1
+                    for (int cc = 0; cc < D / 32; ++cc) {
+                        uint32_t o[32];
+                        const uint32_t oa = x.tmem + lane_addr + 128 + cc * 32;
+                        tmem_ld32(oa, o);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int y = 0; y < 32; ++y)
+                            o[y] = __float_as_uint(__uint_as_float(o[y]) * factor);
+                        tmem_st32(oa, o);
+                    }
+                    tmem_wait_st();
+                }
+                l *= factor;
+                lx *= factor;
+                m_ref = m_new;
+                // P buffer (t & 1) was read by the P V product of tile t - 2
+                if (t >= 2) wait(&x.pv_done[t & 1], static_cast<uint32_t>(((t >> 1) - 1) & 1));
+                if (active) {
+                    unsigned char* prow = smem + C::kOffP + (t & 1) * C::kPBytes;
+#pragma unroll
+                    for (int cc = 0; cc < CW / 8; ++cc) {
+                        float ev[8];
+                        uint32_t w4[4];
+                        float lsum = 0.f, xsum = 0.f;
+#pragma unroll
+                        for (int y = 0; y < 8; ++y) {
+                            // masked keys give 0, also while the row has no finite max yet
+                            const float sk = sv[cc * 8 + y];
+                            ev[y] = sk == kNegInf ? 0.f : ex2(sk - m_ref);
+                            xsum += ev[y];
+                        }
+#pragma unroll
+                        for (int y = 0; y < 4; ++y) {
+                            float ra, rb;
+                            w4[y] = pack_round(ev[2 * y], ev[2 * y + 1], kBF16, ra, rb);
+                            lsum += ra + rb;
+                        }
+                        l += lsum;
+                        lx += xsum;
+                        *reinterpret_cast<uint4*>(prow + swz(r, cb / 8 + cc)) =
+                            make_uint4(w4[0], w4[1], w4[2], w4[3]);
+                    }
+                }
+                fence_proxy_async_smem();
+            }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&x.p_full[t & 1]));
+        }
+
+        // ---- end of piece: merge the replicas, then output or part record
+        const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
+        if (warp_active) {
+            wait(&x.pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+            fence_after();
+        }
+        float M = m_ref, L = l, LX = lx, wgt = 1.f;
+        if constexpr (R > 1) {
+            float* stats = x.scratch;  // [128][3]
+            if (active) {
+                stats[r * 3 + 0] = m_ref;
+                stats[r * 3 + 1] = l;
+                stats[r * 3 + 2] = lx;
+            }
+            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+            if (active) {
+                M = kNegInf;
+#pragma unroll
+                for (int j = 0; j < R; ++j) M = fmaxf(M, stats[(j * RR + g) * 3]);
+                L = 0.f;
+                LX = 0.f;
+#pragma unroll
+                for (int j = 0; j < R; ++j) {
+                    const float wj = rescale(stats[(j * RR + g) * 3], M);
+                    L += wj * stats[(j * RR + g) * 3 + 1];
+                    LX += wj * stats[(j * RR + g) * 3 + 2];
+                }
+                wgt = rescale(m_ref, M);
+            }
+        }
+        const bool writer = active && rep == 0;
+        float* rec = (!whole && writer) ? p.part + ((x.c * 2 + slot) * G + g) * (D + 3) : nullptr;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            if (warp_active) {
+                tmem_ld32(x.tmem + lane_addr + 128 + cc * 32, o);
+                tmem_wait_ld();
+            }
+            if constexpr (R > 1) {
+                if (active)
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) stage[r * 33 + y] = __uint_as_float(o[y]) * wgt;
+                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                if (writer)
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int j = 0; j < R; ++j) a += stage[(j * RR + g) * 33 + y];
+                        o[y] = __float_as_uint(a);
+                    }
+                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+            }
+            if (writer) {
+                if (whole) {
+                    float* dst = p.out + qrow * D + cc * 32;
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) dst[y] = __uint_as_float(o[y]) / L;
+                } else {
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) rec[cc * 32 + y] = __uint_as_float(o[y]);
+                }
+            }
+        }
+        if (writer) {
+            if (whole) {
+                if (p.lse) p.lse[qrow] = (M + log2f(LX)) * kLn2;
+            } else {
+                rec[D] = M;
+                rec[D + 1] = L;
+                rec[D + 2] = LX;
+            }
+        }
+        fence_before();
+        if (!whole) {
+            __threadfence();
+            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+            const long long c_lo = gpart_of(w.start, x.T, x.P);
+            const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
+            const int n = static_cast<int>(c_hi - c_lo + 1);
+            const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+            if (st == 0) {
+                const int prev = atomicAdd(p.tickets + seg, 1);
+                const int last = prev == n - 1;
+                if (last) atomicExch(p.tickets + seg, 0);
+                x.ctl->last = last;
+            }
+            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+            if (x.ctl->last) {
+                __threadfence();
+                const int first_slot = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
+                for (int gg = 0; gg < G; ++gg) {
+                    const long long orow =
+                        static_cast<long long>(w.b) * p.Hq + static_cast<long long>(w.h) * G + gg;
+                    const GSlotAcc acc{p.part, c_lo, first_slot, G, gg, D};
+                    tree_merge(acc, n, D, st, kSoftmaxThreads, x.scratch, kScratchFloats,
+                               kBarSoftmax, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+                }
+            }
+        }
+        named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+        ++pc;
+    } while (gwalk_next(p, *x.ctl, w));
+}
+
+
+template <typename E, int D, int CW>
 __global__ void __launch_bounds__(kGqaThreads, 1)
     td_gqa_kernel(const GqaParams p, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV) {
@@ -501,220 +810,9 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
         __syncwarp();
     } else {
         // --------------------------------------------------------- softmax
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;      // MMA row = query head within the group
-        const bool warp_active = quarter * 32 < G;
-        const bool active = r < G;
-        const int st = tid - 64;                // 0..127 within the softmax warpgroup
-        const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-        const float qscale2 = p.qscale2;
-        long long t = 0;
-        long long pc = 0;
-        bool aborted = false;
-        auto wait = [&](uint64_t* bar, uint32_t par) {
-            if (!aborted && !mbar_wait_bounded(smem_addr(bar), par, abort_flag, p.err,
-                                               TD_DEVERR_WAIT_TIMEOUT))
-                aborted = true;
-        };
-        GWalk w;
-        if (gwalk_first(p, ctl, w)) {
-            do {
-                const long long j0 = (x0 > w.start ? x0 : w.start) - w.start;
-                const long long e = w.start + w.len;
-                const long long j1 = (x1 < e ? x1 : e) - w.start;
-                const long long nt = (j1 - j0 + kTK - 1) / kTK;
-                const bool whole = (j0 == 0 && j1 == w.len);
-                const long long hq = static_cast<long long>(w.h) * G + r;          // query head
-                const long long qrow = static_cast<long long>(w.b) * p.Hq + hq;   // b*Hq + hq
-                // Q rows of this kv head's group, K-major, 128-byte swizzle
-                if (active) {
-                    const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) + qrow * D);
-#pragma unroll
-                    for (int a = 0; a < C::kAtoms; ++a)
-#pragma unroll
-                        for (int cc = 0; cc < 8; ++cc) {
-                            const uint4 v = __ldg(qg + a * 8 + cc);
-                            *reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kM * 128) + swz(r, cc)) = v;
-                        }
-                }
-                fence_proxy_async_smem();
-                fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&q_ready));
-
-                const float slope2 =
-                    (active && p.slopes) ? __ldg(p.slopes + hq) * kLog2e : 0.f;
-                // l: sum of p as rounded for the P V product (normalises O);
-                // lx: sum of the unrounded p (for lse)
-                float m_ref = kNegInf, l = 0.f, lx = 0.f;
-                for (long long i = 0; i < nt; ++i, ++t) {
-                    const long long t0 = j0 + i * kTK;
-                    const int rows = static_cast<int>((j1 - t0) < kTK ? (j1 - t0) : kTK);
-                    wait(&s_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
-                    fence_after();
-                    uint32_t sr[2][32];
-                    if (warp_active) {
-                        const uint32_t sa = tmem + lane_addr + static_cast<uint32_t>((t & 1) * kTK);
-                        tmem_ld32(sa, sr[0]);
-                        tmem_ld32(sa + 32, sr[1]);
-                        tmem_wait_ld();
-                    }
-                    fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&s_empty[t & 1]));
-
-                    if (rows < kTK) {
-                        // keys past the piece end: the tile holds other rows (or padding
-                        // that may not be finite); p is 0 there, and 0 * NaN would poison
-                        // O, so zero those V rows before the P V product reads them
-                        const int stage = static_cast<int>(t % kGqaStages);
-                        unsigned char* vb = smem + C::kOffKV + stage * C::kStageBytes +
-                                            C::kAtoms * C::kKVAtomBytes;
-                        const int n16 = (kTK - rows) * 8 * C::kAtoms;  // 16-B units to clear
-                        for (int i = lane + quarter * 32; i < n16; i += kSoftmaxThreads) {
-                            const int a = i / ((kTK - rows) * 8);
-                            const int rem = i - a * ((kTK - rows) * 8);
-                            const int row = rows + rem / 8, cc = rem % 8;
-                            *reinterpret_cast<uint4*>(vb + a * C::kKVAtomBytes + swz(row, cc)) =
-                                make_uint4(0, 0, 0, 0);
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    if (warp_active) {
-                        float s[kTK];
-                        float mt = kNegInf;
-#pragma unroll
-                        for (int k = 0; k < kTK; ++k) {
-                            const float raw = __uint_as_float(sr[k >> 5][k & 31]);
-                            float v = p.slopes ? fmaf(raw, qscale2,
-                                                      slope2 * static_cast<float>(t0 + k - w.len + 1))
-                                               : raw * qscale2;
-                            v = (k < rows && active) ? v : kNegInf;
-                            s[k] = v;
-                            mt = fmaxf(mt, v);
-                        }
-                        const bool need = active && (m_ref == kNegInf ? mt != kNegInf
-                                                                       : mt > m_ref + kRescaleThreshold);
-                        const float m_new = need ? fmaxf(m_ref, mt) : m_ref;
-                        const float factor = need ? rescale(m_ref, m_new) : 1.f;
-                        if (__any_sync(0xffffffffu, need && i > 0)) {
-                            // O already holds earlier tiles of this piece: scale it
-                            wait(&pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
-                            fence_after();
-#pragma unroll 1
-                            for (int cc = 0; cc < D / 32; ++cc) {
-                                uint32_t o[32];
-                                const uint32_t oa = tmem + lane_addr + 128 + cc * 32;
-                                tmem_ld32(oa, o);
-                                tmem_wait_ld();
-#pragma unroll
-                                for (int x = 0; x < 32; ++x)
-                                    o[x] = __float_as_uint(__uint_as_float(o[x]) * factor);
-                                tmem_st32(oa, o);
-                            }
-                            tmem_wait_st();
-                        }
-                        l *= factor;
-                        lx *= factor;
-                        m_ref = m_new;
-                        // P buffer (t & 1) was read by the P V product of tile t - 2
-                        if (t >= 2)
-                            wait(&pv_done[t & 1], static_cast<uint32_t>(((t >> 1) - 1) & 1));
-                        if (active) {
-                            unsigned char* prow = smem + C::kOffP + (t & 1) * C::kPBytes;
-#pragma unroll
-                            for (int cc = 0; cc < 8; ++cc) {
-                                float e[8];
-                                uint32_t w4[4];
-                                float lsum = 0.f, xsum = 0.f;
-#pragma unroll
-                                for (int x = 0; x < 8; ++x) {
-                                    e[x] = ex2(s[cc * 8 + x] - m_ref);
-                                    xsum += e[x];
-                                }
-#pragma unroll
-                                for (int x = 0; x < 4; ++x) {
-                                    float ra, rb;
-                                    w4[x] = pack_round(e[2 * x], e[2 * x + 1], kBF16, ra, rb);
-                                    lsum += ra + rb;
-                                }
-                                l += lsum;
-                                lx += xsum;
-                                *reinterpret_cast<uint4*>(prow + swz(r, cc)) =
-                                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
-                            }
-                        }
-                        fence_proxy_async_smem();
-                    }
-                    fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_addr(&p_full[t & 1]));
-                }
-
-                // ---- end of piece: O rows of this group
-                float* rec = nullptr;
-                const int slot = pc == 0 ? 0 : 1;  // first piece of the CTA uses slot 0
-                if (warp_active) {
-                    wait(&pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
-                    fence_after();
-                    if (!whole) rec = p.part + ((c * 2 + slot) * G + r) * (D + 3);
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld32(tmem + lane_addr + 128 + cc * 32, o);
-                        tmem_wait_ld();
-                        if (active) {
-                            if (whole) {
-                                float* dst = p.out + qrow * D + cc * 32;
-#pragma unroll
-                                for (int x = 0; x < 32; ++x) dst[x] = __uint_as_float(o[x]) / l;
-                            } else {
-#pragma unroll
-                                for (int x = 0; x < 32; ++x) rec[cc * 32 + x] = __uint_as_float(o[x]);
-                            }
-                        }
-                    }
-                    if (active) {
-                        if (whole) {
-                            if (p.lse) p.lse[qrow] = (m_ref + log2f(lx)) * kLn2;
-                        } else {
-                            rec[D] = m_ref;
-                            rec[D + 1] = l;
-                            rec[D + 2] = lx;
-                        }
-                    }
-                    fence_before();
-                }
-                if (!whole) {
-                    __threadfence();
-                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-                    const long long c_lo = gpart_of(w.start, T, P);
-                    const long long c_hi = gpart_of(w.start + w.len - 1, T, P);
-                    const int n = static_cast<int>(c_hi - c_lo + 1);
-                    const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
-                    if (st == 0) {
-                        const int prev = atomicAdd(p.tickets + seg, 1);
-                        const int last = prev == n - 1;
-                        if (last) atomicExch(p.tickets + seg, 0);
-                        ctl.last = last;
-                    }
-                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-                    if (ctl.last) {
-                        __threadfence();
-                        const int first_slot = gpart_start(c_lo, T, P) < w.start ? 1 : 0;
-                        for (int g = 0; g < G; ++g) {
-                            const long long orow = static_cast<long long>(w.b) * p.Hq +
-                                                   static_cast<long long>(w.h) * G + g;
-                            const GSlotAcc acc{p.part, c_lo, first_slot, G, g, D};
-                            tree_merge(acc, n, D, st, kSoftmaxThreads, scratch, kScratchFloats,
-                                       kBarSoftmax, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
-                        }
-                    }
-                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-                }
-                ++pc;
-            } while (gwalk_next(p, ctl, w));
-        }
+        const SmCtx sx{smem, scratch, s_full, s_empty, p_full, pv_done, &q_ready, &ctl, abort_flag,
+                       tmem, T, x0, x1, P, c, warp, lane, tid};
+        softmax_role<E, D, CW>(p, sx);
     }
 
     fence_before();
@@ -726,11 +824,11 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
     }
 }
 
-template <typename E, int D>
+template <typename E, int D, int CW>
 cudaError_t launch_gqa_t(int device, const GqaParams& p, const CUtensorMap& mk,
                          const CUtensorMap& mv, cudaStream_t s) {
     using C = GCfg<D>;
-    auto kern = td_gqa_kernel<E, D>;
+    auto kern = td_gqa_kernel<E, D, CW>;
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
     if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
@@ -743,6 +841,17 @@ cudaError_t launch_gqa_t(int device, const GqaParams& p, const CUtensorMap& mk,
     return cudaGetLastError();
 }
 
+
+template <typename E, int D>
+cudaError_t launch_gqa_g(int device, const GqaParams& p, const CUtensorMap& mk,
+                         const CUtensorMap& mv, cudaStream_t s) {
+    // key columns per replica of the query rows: 4 replicas while G fits a
+    // TMEM lane quarter, 2 while it fits half, else 1
+    if (p.G <= 32) return launch_gqa_t<E, D, 16>(device, p, mk, mv, s);
+    if (p.G <= 64) return launch_gqa_t<E, D, 32>(device, p, mk, mv, s);
+    return launch_gqa_t<E, D, 64>(device, p, mk, mv, s);
+}
+
 }  // namespace
 
 size_t gqa_smem_bytes(int D) {
@@ -752,11 +861,11 @@ size_t gqa_smem_bytes(int D) {
 cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const CUtensorMap& mk,
                        const CUtensorMap& mv, cudaStream_t s) {
     if (dtype == kBF16) {
-        if (D == 64) return launch_gqa_t<__nv_bfloat16, 64>(device, p, mk, mv, s);
-        if (D == 128) return launch_gqa_t<__nv_bfloat16, 128>(device, p, mk, mv, s);
+        if (D == 64) return launch_gqa_g<__nv_bfloat16, 64>(device, p, mk, mv, s);
+        if (D == 128) return launch_gqa_g<__nv_bfloat16, 128>(device, p, mk, mv, s);
     } else if (dtype == kF16) {
-        if (D == 64) return launch_gqa_t<__half, 64>(device, p, mk, mv, s);
-        if (D == 128) return launch_gqa_t<__half, 128>(device, p, mk, mv, s);
+        if (D == 64) return launch_gqa_g<__half, 64>(device, p, mk, mv, s);
+        if (D == 128) return launch_gqa_g<__half, 128>(device, p, mk, mv, s);
     }
     return cudaErrorInvalidValue;
 }

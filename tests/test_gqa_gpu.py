@@ -113,3 +113,14 @@ def test_gqa_rejects_unsupported():
     inp = make_gqa_inputs(w, 4, DEV)
     with pytest.raises(td.TreeDecError, match="INVALID"):
         td.decode_gqa(inp["q"], inp["k"], inp["v"])
+
+
+def test_gqa_short_pieces_leave_replica_slices_empty():
+    """Pieces shorter than a tile (a part that ends one sequence after a few
+    keys and starts the next) leave some key-column slices with no key."""
+    w = Workload("gqa_short", torch.bfloat16, 3, 8, 128, 70, alibi=True, seed=900)
+    for parts in (4, 5, 7, 11, 13, 50, 210):
+        run_and_check(w, 2, parts=parts)
+    w = Workload("gqa_tiny", torch.float16, 4, 4, 64, 5, seed=901)
+    for parts in (1, 3, 20):
+        run_and_check(w, 1, parts=parts)
