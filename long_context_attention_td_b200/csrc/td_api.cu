@@ -270,9 +270,14 @@ td_status decode_impl(const Req& r) {
 // ------------------------------------------------------------- grouped-query
 
 constexpr int kGqaCtasPerSm = 1;
+// parts-per-sequence x group size above which the merge runs as its own kernel
+constexpr long long kGqaSeparateMerge = 128;
+
+// [error word][tickets][segment descriptors: 3 int32 each][part records]
+size_t gqa_desc_region(long long BHkv) { return align_up(static_cast<size_t>(BHkv) * 12, 256); }
 
 size_t gqa_ws_bytes_for(long long BHkv, int G, int D, long long parts) {
-    return td::kErrRegion + ticket_region(BHkv) +
+    return td::kErrRegion + ticket_region(BHkv) + gqa_desc_region(BHkv) +
            static_cast<size_t>(parts) * 2 * static_cast<size_t>(G) *
                static_cast<size_t>(D + 3) * sizeof(float);
 }
@@ -419,8 +424,17 @@ td_status gqa_impl(const GqaReq& r) {
     p.qscale2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(r.D)));
     p.err = reinterpret_cast<int*>(base);
     p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
-    p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BHkv));
-    return cuda_status(td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
+    p.seg_desc = reinterpret_cast<int*>(base + td::kErrRegion + ticket_region(BHkv));
+    p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BHkv) +
+                                      gqa_desc_region(BHkv));
+    // The last CTA of a sequence merges its parts itself when that is a small
+    // job; when many CTAs share a sequence and many query heads share it, a
+    // second kernel spreads the merge over one CTA per (sequence, query head).
+    const long long per_seg = (P + BHkv - 1) / BHkv + 1;  // parts touching a sequence
+    p.fused_merge = per_seg * G < kGqaSeparateMerge ? 1 : 0;
+    st = cuda_status(td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
+    if (st != TD_OK || p.fused_merge) return st;
+    return cuda_status(td::launch_gqa_combine(r.D, p, r.stream));
 }
 
 }  // namespace

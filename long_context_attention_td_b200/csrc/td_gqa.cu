@@ -542,7 +542,18 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
             }
         }
         fence_before();
-        if (!whole) {
+        if (!p.fused_merge) {
+            // the CTA holding the sequence's first key describes its parts for
+            // the combine kernel (one part: already written, nothing to merge)
+            if (j0 == 0 && st == 0) {
+                const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+                const long long c_lo = gpart_of(w.start, x.T, x.P);
+                const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
+                p.seg_desc[seg * 3 + 0] = static_cast<int>(c_lo);
+                p.seg_desc[seg * 3 + 1] = static_cast<int>(c_hi - c_lo + 1);
+                p.seg_desc[seg * 3 + 2] = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
+            }
+        } else if (!whole) {
             __threadfence();
             named_bar_sync(kBarSoftmax, kSoftmaxThreads);
             const long long c_lo = gpart_of(w.start, x.T, x.P);
@@ -679,6 +690,8 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
             for (int i = tid; i < p.Hq * D; i += kGqaThreads) p.out[b * p.Hq * D + i] = 0.f;
             if (p.lse)
                 for (int h = tid; h < p.Hq; h += kGqaThreads) p.lse[b * p.Hq + h] = kNegInf;
+            if (!p.fused_merge)
+                for (int h = tid; h < p.Hkv; h += kGqaThreads) p.seg_desc[(b * p.Hkv + h) * 3 + 1] = 0;
         }
     }
     fence_before();
@@ -853,6 +866,31 @@ cudaError_t launch_gqa_g(int device, const GqaParams& p, const CUtensorMap& mk,
 }
 
 }  // namespace
+
+// One CTA per (sequence, query head) of the split sequences: the gist's
+// global max, renormalisation and sums over the sequence's part records.
+__global__ void __launch_bounds__(kSoftmaxThreads) td_gqa_combine_kernel(const GqaParams p, int D) {
+    __shared__ float scratch[kScratchFloats];
+    const long long seg = blockIdx.x;
+    const int g = blockIdx.y;
+    const int n = p.seg_desc[seg * 3 + 1];
+    if (n <= 1) return;
+    const long long c_lo = p.seg_desc[seg * 3 + 0];
+    const int first_slot = p.seg_desc[seg * 3 + 2];
+    const long long b = seg / p.Hkv, h = seg % p.Hkv;
+    const long long orow = b * p.Hq + h * p.G + g;
+    const GSlotAcc acc{p.part, c_lo, first_slot, p.G, g, D};
+    tree_merge(acc, n, D, static_cast<int>(threadIdx.x), kSoftmaxThreads, scratch, kScratchFloats,
+               1, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+}
+
+cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s) {
+    const long long segs = static_cast<long long>(p.B) * p.Hkv;
+    if (segs > 0x7fffffffLL || p.G > 65535) return cudaErrorInvalidValue;
+    dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(p.G));
+    td_gqa_combine_kernel<<<grid, kSoftmaxThreads, 0, s>>>(p, D);
+    return cudaGetLastError();
+}
 
 size_t gqa_smem_bytes(int D) {
     return D == 64 ? GCfg<64>::kSmem : D == 128 ? GCfg<128>::kSmem : 0;

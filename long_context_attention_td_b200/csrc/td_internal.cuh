@@ -75,12 +75,16 @@ struct GqaParams {
     float qscale2;           // D^-1/2 * log2(e)
     float* part;             // part records [P][2][G][D + 3]
     int* tickets;            // [B * Hkv]
+    int* seg_desc;           // [B * Hkv][3]: first part, parts, slot of the first part
+    int fused_merge;         // 1: last CTA merges (ticket); 0: td_gqa_combine merges
     int* err;
 };
 size_t gqa_smem_bytes(int D);
 // K and V tensor maps: 2-D [B*Hkv*N rows, D columns], box {64, 64}, 128-byte swizzle.
 cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const CUtensorMap& mk,
                        const CUtensorMap& mv, cudaStream_t s);
+// Merge the part records of every split sequence (p.fused_merge == 0).
+cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s);
 
 // Dynamic shared memory of the split-KV kernel for (dtype, D).
 size_t partial_smem_bytes(int dtype, int D);
