@@ -12,17 +12,19 @@
 // over the CTAs, exactly as in td_partial; pieces of a sequence cut across CTAs
 // are merged by the last CTA to finish (atomic ticket), per query head.
 //
-// One CTA per SM, 6 warps:
+// One CTA per SM, 10 warps:
 //   warp 0      TMA producer: K and V tiles of 64 keys, 2-D tensor-map loads
 //               with 128-byte swizzle (one box per 64 columns of D), 4 stages;
-//   warp 1      allocates 256 TMEM columns and issues the MMAs from one lane:
-//               S(t) = Q K(t)^T into one of two S buffers, then O += P(t) V(t)
-//               into the O accumulator, completion signalled by tcgen05.commit;
-//   warps 2-5   softmax warpgroup (warp w reads TMEM lanes 32*(w%4)..+31, one
-//               query head per lane): read S, scale, ALiBi term, row max,
-//               p = 2^(s - m) rounded to the input type and written to shared
-//               memory as the A operand of the P V product; at the end of a
-//               piece read O and write the output or a part record.
+//   warp 1      allocates 512 TMEM columns and issues the MMAs from one lane:
+//               S(t) = Q K(t)^T into S buffer t%2, O(t%2) += P(t) V(t), with
+//               completion signalled by tcgen05.commit;
+//   warps 2-5   softmax warpgroup 0 (even tiles), warps 6-9 warpgroup 1 (odd
+//               tiles); warp w reads TMEM lanes 32*(w%4)..+31.  Each group keeps
+//               its own running max and O accumulator, so one group's latency
+//               chain (read S, exponentials, write P) overlaps the other's.  The
+//               query rows are replicated across the lane quarters (see
+//               softmax_role) and every (group, replica) is merged at the end of
+//               a piece, which then gives the output or a part record.
 // The running max m of a row is only moved when a tile's max exceeds it by
 // more than 8 (log2 units); O in TMEM is rescaled then, and p <= 2^8 otherwise.
 #include <cuda.h>
@@ -43,9 +45,9 @@ using namespace dev;
 constexpr int kTK = 64;            // keys per tile
 constexpr int kM = 128;            // MMA rows (query heads, padded)
 constexpr int kGqaStages = 4;      // K/V pipeline depth
-constexpr int kGqaThreads = 192;   // 6 warps
-constexpr int kSoftmaxThreads = 128;
-constexpr int kTmemCols = 256;     // S0 [0,64) S1 [64,128) O [128,128+D)
+constexpr int kGqaThreads = 320;   // 10 warps
+constexpr int kSoftmaxThreads = 128;  // one softmax warpgroup
+constexpr int kTmemCols = 512;     // S0 [0,64) S1 [64,128) O0 [128,256) O1 [256,384)
 constexpr int kScratchFloats = 1024;
 constexpr float kRescaleThreshold = 8.f;  // log2 units
 
@@ -266,7 +268,8 @@ __device__ __forceinline__ long long gpart_of(long long x, long long T, long lon
     return ((x + 1) * P - 1) / T;
 }
 
-constexpr int kBarSoftmax = 1;
+constexpr int kBarSoftmax = 1;  // named barrier of softmax warpgroup 0
+constexpr int kBarGroups = 2;   // named barrier of both softmax warpgroups
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
     asm volatile(
@@ -305,19 +308,23 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
     constexpr int R = kTK / CW;   // replicas
     constexpr int RR = kM / R;    // MMA rows per replica
     const int G = p.G;
+    const int grp = (x.warp - 2) >> 2;    // 0: even tiles, 1: odd tiles
     const int quarter = x.warp & 3;
     const int r = quarter * 32 + x.lane;  // MMA row (TMEM lane)
     const int rep = r / RR;               // replica: key-column slice of each tile
     const int g = r - rep * RR;           // query head within the group
     const bool warp_active = ((quarter * 32) % RR) < G;
     const bool active = g < G;
-    const int st = x.tid - 64;            // 0..127 within the warpgroup
+    const int st = (x.tid - 64) & (kSoftmaxThreads - 1);  // 0..127 within the warpgroup
     const int lane = x.lane;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t o_col = 128u + 128u * static_cast<uint32_t>(grp);  // this group's O
     const int cb = rep * CW;              // first key column of this replica
     const float qscale2 = p.qscale2;
     unsigned char* smem = x.smem;
     float* stage = reinterpret_cast<float*>(smem + C::kOffStage);
+    float* stats = x.scratch;             // group 0: merged (m, l, lx) per row
+    float* stats1 = x.scratch + 3 * kM;   // group 1's (m, l, lx) per row
     long long t = 0;
     long long pc = 0;
     bool aborted = false;
@@ -337,17 +344,19 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
         const long long hq = static_cast<long long>(w.h) * G + g;          // query head
         const long long qrow = static_cast<long long>(w.b) * p.Hq + hq;   // b*Hq + hq
         // Q rows of this kv head's group (each replica a copy), K-major SW128
-        if (active) {
-            const uint4* qg =
-                reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) + qrow * D);
+        if (grp == 0) {
+            if (active) {
+                const uint4* qg =
+                    reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) + qrow * D);
 #pragma unroll
-            for (int a = 0; a < C::kAtoms; ++a)
+                for (int a = 0; a < C::kAtoms; ++a)
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    *reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kM * 128) + swz(r, cc)) =
-                        __ldg(qg + a * 8 + cc);
+                    for (int cc = 0; cc < 8; ++cc)
+                        *reinterpret_cast<uint4*>(smem + C::kOffQ + a * (kM * 128) + swz(r, cc)) =
+                            __ldg(qg + a * 8 + cc);
+            }
+            fence_proxy_async_smem();
         }
-        fence_proxy_async_smem();
         fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(x.q_ready));
@@ -356,15 +365,17 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
         // l: sum of p as rounded for the P V product (normalises O);
         // lx: sum of the unrounded p (for lse)
         float m_ref = kNegInf, l = 0.f, lx = 0.f;
+        long long last_own = -1;
         for (long long i = 0; i < nt; ++i, ++t) {
+            if (static_cast<int>(t & 1) != grp) continue;
+            last_own = t;
             const long long t0 = j0 + i * kTK;
             const int rows = static_cast<int>((j1 - t0) < kTK ? (j1 - t0) : kTK);
-            wait(&x.s_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
+            wait(&x.s_full[grp], static_cast<uint32_t>((t >> 1) & 1));
             fence_after();
             uint32_t sr[CW];
             if (warp_active) {
-                const uint32_t sa =
-                    x.tmem + lane_addr + static_cast<uint32_t>((t & 1) * kTK + cb);
+                const uint32_t sa = x.tmem + lane_addr + static_cast<uint32_t>(grp * kTK + cb);
                 if constexpr (CW == 16) {
                     tmem_ld16(sa, sr);
                 } else {
@@ -376,7 +387,7 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
             }
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[t & 1]));
+            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[grp]));
 
             if (rows < kTK) {
                 // keys past the piece end: the tile holds other rows (or padding
@@ -394,6 +405,10 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
                 }
                 fence_proxy_async_smem();
             }
+            // the group's previous P V product (tile t - 2) read this P buffer
+            // and wrote this O accumulator
+            if (t >= 2) wait(&x.pv_done[grp], static_cast<uint32_t>(((t >> 1) - 1) & 1));
+            fence_after();
             if (warp_active) {
                 float sv[CW];
                 float mt = kNegInf;
@@ -414,12 +429,10 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
                 const float factor = need ? rescale(m_ref, m_new) : 1.f;
                 if (__any_sync(0xffffffffu, need && m_ref != kNegInf)) {
                     // O already holds earlier tiles of this piece: scale it
-                    wait(&x.pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
-                    fence_after();
 #pragma unroll 1
                     for (int cc = 0; cc < D / 32; ++cc) {
                         uint32_t o[32];
-                        const uint32_t oa = x.tmem + lane_addr + 128 + cc * 32;
+                        const uint32_t oa = x.tmem + lane_addr + o_col + cc * 32;
                         tmem_ld32(oa, o);
                         tmem_wait_ld();
 #pragma unroll
@@ -432,10 +445,8 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
                 l *= factor;
                 lx *= factor;
                 m_ref = m_new;
-                // P buffer (t & 1) was read by the P V product of tile t - 2
-                if (t >= 2) wait(&x.pv_done[t & 1], static_cast<uint32_t>(((t >> 1) - 1) & 1));
                 if (active) {
-                    unsigned char* prow = smem + C::kOffP + (t & 1) * C::kPBytes;
+                    unsigned char* prow = smem + C::kOffP + grp * C::kPBytes;
 #pragma unroll
                     for (int cc = 0; cc < CW / 8; ++cc) {
                         float ev[8];
@@ -464,126 +475,158 @@ __device__ __forceinline__ void softmax_role(const GqaParams& p, const SmCtx& x)
             }
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&x.p_full[t & 1]));
+            if (lane == 0) mbar_arrive(smem_addr(&x.p_full[grp]));
         }
 
-        // ---- end of piece: merge the replicas, then output or part record
-        const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
-        if (warp_active) {
-            wait(&x.pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+        // ---- end of piece: the group's last P V product must be complete
+        if (last_own >= 0 && warp_active) {
+            wait(&x.pv_done[grp], static_cast<uint32_t>((last_own >> 1) & 1));
             fence_after();
         }
-        float M = m_ref, L = l, LX = lx, wgt = 1.f;
-        if constexpr (R > 1) {
-            float* stats = x.scratch;  // [128][3]
+        if (grp == 1) {
+            // hand this group's row state to group 0, which merges and writes
             if (active) {
-                stats[r * 3 + 0] = m_ref;
-                stats[r * 3 + 1] = l;
-                stats[r * 3 + 2] = lx;
+                stats1[r * 3 + 0] = m_ref;
+                stats1[r * 3 + 1] = l;
+                stats1[r * 3 + 2] = lx;
             }
-            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+            fence_before();
+            named_bar_sync(kBarGroups, 2 * kSoftmaxThreads);
+        } else {
+            named_bar_sync(kBarGroups, 2 * kSoftmaxThreads);
+            fence_after();
+            // this row's state over both groups
+            float m1 = kNegInf, l1 = 0.f, lx1 = 0.f;
             if (active) {
-                M = kNegInf;
-#pragma unroll
-                for (int j = 0; j < R; ++j) M = fmaxf(M, stats[(j * RR + g) * 3]);
-                L = 0.f;
-                LX = 0.f;
-#pragma unroll
-                for (int j = 0; j < R; ++j) {
-                    const float wj = rescale(stats[(j * RR + g) * 3], M);
-                    L += wj * stats[(j * RR + g) * 3 + 1];
-                    LX += wj * stats[(j * RR + g) * 3 + 2];
-                }
-                wgt = rescale(m_ref, M);
+                m1 = stats1[r * 3 + 0];
+                l1 = stats1[r * 3 + 1];
+                lx1 = stats1[r * 3 + 2];
             }
-        }
-        const bool writer = active && rep == 0;
-        float* rec = (!whole && writer) ? p.part + ((x.c * 2 + slot) * G + g) * (D + 3) : nullptr;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            if (warp_active) {
-                tmem_ld32(x.tmem + lane_addr + 128 + cc * 32, o);
-                tmem_wait_ld();
-            }
+            const float Mr = fmaxf(m_ref, m1);
+            const float w0 = rescale(m_ref, Mr), w1 = rescale(m1, Mr);
+            const bool use1 = m1 != kNegInf;  // group 1's O holds this piece's tiles
+            const bool any1 = __any_sync(0xffffffffu, active && use1);
+            float M = Mr, L = w0 * l + w1 * l1, LX = w0 * lx + w1 * lx1, wgt = 1.f;
             if constexpr (R > 1) {
-                if (active)
-#pragma unroll
-                    for (int y = 0; y < 32; ++y) stage[r * 33 + y] = __uint_as_float(o[y]) * wgt;
                 named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-                if (writer)
+                if (active) {
+                    stats[r * 3 + 0] = M;
+                    stats[r * 3 + 1] = L;
+                    stats[r * 3 + 2] = LX;
+                }
+                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                if (active) {
+                    M = kNegInf;
+#pragma unroll
+                    for (int j = 0; j < R; ++j) M = fmaxf(M, stats[(j * RR + g) * 3]);
+                    L = 0.f;
+                    LX = 0.f;
+#pragma unroll
+                    for (int j = 0; j < R; ++j) {
+                        const float wj = rescale(stats[(j * RR + g) * 3], M);
+                        L += wj * stats[(j * RR + g) * 3 + 1];
+                        LX += wj * stats[(j * RR + g) * 3 + 2];
+                    }
+                    wgt = rescale(Mr, M);
+                }
+            }
+            const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
+            const bool writer = active && rep == 0;
+            float* rec =
+                (!whole && writer) ? p.part + ((x.c * 2 + slot) * G + g) * (D + 3) : nullptr;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                if (warp_active) {
+                    uint32_t o1[32];
+                    tmem_ld32(x.tmem + lane_addr + 128 + cc * 32, o);
+                    if (any1) tmem_ld32(x.tmem + lane_addr + 256 + cc * 32, o1);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int y = 0; y < 32; ++y) {
-                        float a = 0.f;
-#pragma unroll
-                        for (int j = 0; j < R; ++j) a += stage[(j * RR + g) * 33 + y];
-                        o[y] = __float_as_uint(a);
+                        float v = __uint_as_float(o[y]) * w0;
+                        if (any1 && use1) v = fmaf(w1, __uint_as_float(o1[y]), v);
+                        o[y] = __float_as_uint(v);
                     }
-                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                }
+                if constexpr (R > 1) {
+                    if (active)
+#pragma unroll
+                        for (int y = 0; y < 32; ++y) stage[r * 33 + y] = __uint_as_float(o[y]) * wgt;
+                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                    if (writer)
+#pragma unroll
+                        for (int y = 0; y < 32; ++y) {
+                            float a = 0.f;
+#pragma unroll
+                            for (int j = 0; j < R; ++j) a += stage[(j * RR + g) * 33 + y];
+                            o[y] = __float_as_uint(a);
+                        }
+                    named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                }
+                if (writer) {
+                    if (whole) {
+                        float* dst = p.out + qrow * D + cc * 32;
+#pragma unroll
+                        for (int y = 0; y < 32; ++y) dst[y] = __uint_as_float(o[y]) / L;
+                    } else {
+#pragma unroll
+                        for (int y = 0; y < 32; ++y) rec[cc * 32 + y] = __uint_as_float(o[y]);
+                    }
+                }
             }
             if (writer) {
                 if (whole) {
-                    float* dst = p.out + qrow * D + cc * 32;
-#pragma unroll
-                    for (int y = 0; y < 32; ++y) dst[y] = __uint_as_float(o[y]) / L;
+                    if (p.lse) p.lse[qrow] = (M + log2f(LX)) * kLn2;
                 } else {
-#pragma unroll
-                    for (int y = 0; y < 32; ++y) rec[cc * 32 + y] = __uint_as_float(o[y]);
+                    rec[D] = M;
+                    rec[D + 1] = L;
+                    rec[D + 2] = LX;
                 }
             }
-        }
-        if (writer) {
-            if (whole) {
-                if (p.lse) p.lse[qrow] = (M + log2f(LX)) * kLn2;
-            } else {
-                rec[D] = M;
-                rec[D + 1] = L;
-                rec[D + 2] = LX;
-            }
-        }
-        fence_before();
-        if (!p.fused_merge) {
-            // the CTA holding the sequence's first key describes its parts for
-            // the combine kernel (one part: already written, nothing to merge)
-            if (j0 == 0 && st == 0) {
-                const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+            fence_before();
+            if (!p.fused_merge) {
+                // the CTA holding the sequence's first key describes its parts for
+                // the combine kernel (one part: already written, nothing to merge)
+                if (j0 == 0 && st == 0) {
+                    const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+                    const long long c_lo = gpart_of(w.start, x.T, x.P);
+                    const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
+                    p.seg_desc[seg * 3 + 0] = static_cast<int>(c_lo);
+                    p.seg_desc[seg * 3 + 1] = static_cast<int>(c_hi - c_lo + 1);
+                    p.seg_desc[seg * 3 + 2] = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
+                }
+            } else if (!whole) {
+                __threadfence();
+                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
                 const long long c_lo = gpart_of(w.start, x.T, x.P);
                 const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
-                p.seg_desc[seg * 3 + 0] = static_cast<int>(c_lo);
-                p.seg_desc[seg * 3 + 1] = static_cast<int>(c_hi - c_lo + 1);
-                p.seg_desc[seg * 3 + 2] = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
-            }
-        } else if (!whole) {
-            __threadfence();
-            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-            const long long c_lo = gpart_of(w.start, x.T, x.P);
-            const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
-            const int n = static_cast<int>(c_hi - c_lo + 1);
-            const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
-            if (st == 0) {
-                const int prev = atomicAdd(p.tickets + seg, 1);
-                const int last = prev == n - 1;
-                if (last) atomicExch(p.tickets + seg, 0);
-                x.ctl->last = last;
-            }
-            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
-            if (x.ctl->last) {
-                __threadfence();
-                const int first_slot = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
-                for (int gg = 0; gg < G; ++gg) {
-                    const long long orow =
-                        static_cast<long long>(w.b) * p.Hq + static_cast<long long>(w.h) * G + gg;
-                    const GSlotAcc acc{p.part, c_lo, first_slot, G, gg, D};
-                    tree_merge(acc, n, D, st, kSoftmaxThreads, x.scratch, kScratchFloats,
-                               kBarSoftmax, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+                const int n = static_cast<int>(c_hi - c_lo + 1);
+                const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+                if (st == 0) {
+                    const int prev = atomicAdd(p.tickets + seg, 1);
+                    const int last = prev == n - 1;
+                    if (last) atomicExch(p.tickets + seg, 0);
+                    x.ctl->last = last;
+                }
+                named_bar_sync(kBarSoftmax, kSoftmaxThreads);
+                if (x.ctl->last) {
+                    __threadfence();
+                    const int first_slot = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
+                    for (int gg = 0; gg < G; ++gg) {
+                        const long long orow = static_cast<long long>(w.b) * p.Hq +
+                                               static_cast<long long>(w.h) * G + gg;
+                        const GSlotAcc acc{p.part, c_lo, first_slot, G, gg, D};
+                        tree_merge(acc, n, D, st, kSoftmaxThreads, x.scratch, kScratchFloats,
+                                   kBarSoftmax, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+                    }
                 }
             }
+            named_bar_sync(kBarSoftmax, kSoftmaxThreads);
         }
-        named_bar_sync(kBarSoftmax, kSoftmaxThreads);
         ++pc;
     } while (gwalk_next(p, *x.ctl, w));
 }
-
 
 template <typename E, int D, int CW>
 __global__ void __launch_bounds__(kGqaThreads, 1)
@@ -617,7 +660,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
             mbar_init(smem_addr(&p_full[s]), 4);
             mbar_init(smem_addr(&pv_done[s]), 1);
         }
-        mbar_init(smem_addr(&q_ready), 4);
+        mbar_init(smem_addr(&q_ready), 8);
         fence_barrier_init();
         ctl.abort = 0;
         ctl.last = 0;
@@ -632,7 +675,7 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
         // Q and both P buffers start at zero (rows >= G stay zero)
         uint4* z = reinterpret_cast<uint4*>(smem + C::kOffQ);
         const int n16 = (C::kQBytes + 2 * C::kPBytes) / 16;
-        for (int i = tid - 64; i < n16; i += kSoftmaxThreads) z[i] = make_uint4(0, 0, 0, 0);
+        for (int i = tid - 64; i < n16; i += kGqaThreads - 64) z[i] = make_uint4(0, 0, 0, 0);
         fence_proxy_async_smem();
     }
     if (p.seqlens == nullptr) {
@@ -793,32 +836,36 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
                     wait(&q_ready, static_cast<uint32_t>(pc & 1));
                     fence_after();
                     issue_S(t);
+                    if (nt > 1) issue_S(t + 1);
                     for (long long i = 0; i < nt; ++i, ++t) {
-                        if (i + 1 < nt) issue_S(t + 1);
                         wait(&p_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
                         fence_after();
                         const int stage = static_cast<int>(t % kGqaStages);
                         const uint32_t vb = sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtomBytes;
                         const uint32_t pb = sP + static_cast<uint32_t>((t & 1) * C::kPBytes);
+                        const uint32_t dO = tmem + 128 + static_cast<uint32_t>((t & 1) * 128);
 #pragma unroll
                         for (int kk = 0; kk < kTK / 16; ++kk) {
                             const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
                             const uint64_t b =
                                 smem_desc_sw128(vb + kk * 2048, C::kKVAtomBytes, 1024);
-                            umma_f16(tmem + 128, a, b, idO, (i > 0 || kk > 0) ? 1u : 0u);
+                            // each group's first tile of the piece starts its accumulator
+                            umma_f16(dO, a, b, idO, (i > 1 || kk > 0) ? 1u : 0u);
                         }
                         umma_commit(smem_addr(&pv_done[t & 1]));
                         umma_commit(smem_addr(&kv_empty[stage]));
                         last_pv = t;
+                        if (i + 2 < nt) issue_S(t + 2);
                     }
                     ++pc;
                 } while (gwalk_next(p, ctl, w));
             }
             // every MMA must be complete before the CTA frees TMEM
-            if (last_pv >= 0)
-                mbar_wait_bounded(smem_addr(&pv_done[last_pv & 1]),
-                                  static_cast<uint32_t>((last_pv >> 1) & 1), nullptr, p.err,
-                                  TD_DEVERR_WAIT_TIMEOUT);
+            for (long long tl = last_pv - 1; tl <= last_pv; ++tl)
+                if (tl >= 0)
+                    mbar_wait_bounded(smem_addr(&pv_done[tl & 1]),
+                                      static_cast<uint32_t>((tl >> 1) & 1), nullptr, p.err,
+                                      TD_DEVERR_WAIT_TIMEOUT);
         }
         __syncwarp();
     } else {
