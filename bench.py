@@ -180,9 +180,35 @@ def barrier():
 
 # -------------------------------------------------------------- CPU oracle
 
+def oracle_rate_gqa(inp, w, budget_s, min_s=0.0, threads=0):
+    """The same for grouped-query workloads: every query head of batch 0 over
+    the first keys of its kv head, shortened to the time budget."""
+    import oracle
+    cores = os.cpu_count() or 1
+    threads = threads or cores
+    Hkv = w.kv_heads
+    nk = max(1024, min(w.N, int(budget_s * 0.5e9 * min(threads, w.H) / (2 * w.D * w.elt * w.H))))
+    q = inp["q"][:1].cpu()
+    k = inp["k"][:1, :, :nk].cpu().contiguous()
+    v = inp["v"][:1, :, :nk].cpu().contiguous()
+    bytes_once = 2 * Hkv * nk * w.D * w.elt
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.full_gqa(q, k, v, threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            break
+    desc = ("%d query heads over %d kv heads x %d keys (%s, D=%d), %d pass(es), %d thread(s)"
+            % (w.H, Hkv, nk, DTYPE_NAME[w.dtype], w.D, passes, min(threads, w.H)))
+    return bytes_once * passes / dt / 1e9, min(threads, w.H), desc, dt
+
+
 def oracle_rate(inp, w, budget_s, min_s=0.0, threads=0):
     """Time the fp64 oracle on (b,h) rows of a host copy of the workload;
     returns (GB/s, threads used, description, seconds)."""
+    if w.kv_heads and w.kv_heads != w.H:
+        return oracle_rate_gqa(inp, w, budget_s, min_s, threads)
     import oracle
     B, H = w.B, w.H
     cores = os.cpu_count() or 1
@@ -247,11 +273,19 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     B, H, D, N = w.B, w.H, w.D, w.N
     total_keys = kv_lengths(w, inp["seqlens_host"])
-    parts = td.plan_parts(B, H, N, D, w.dtype, n_split,
-                          total_keys if inp["seqlens"] is not None else -1)
+    gqa = bool(w.kv_heads) and w.kv_heads != w.H
+    if gqa:
+        parts = td.plan_parts_gqa(B, H, w.kv_heads, N, D, w.dtype, n_split,
+                                  total_keys if inp["seqlens"] is not None else -1)
+    else:
+        parts = td.plan_parts(B, H, N, D, w.dtype, n_split,
+                              total_keys if inp["seqlens"] is not None else -1)
 
     def step():
-        if inp["seqlens"] is not None:
+        if gqa:
+            td.decode_gqa(q, k, v, seqlens=inp["seqlens"], seqlens_host=inp["seqlens_host"],
+                          slopes=inp["slopes"], n_split=n_split, out=out, lse=lse, stream=stream)
+        elif inp["seqlens"] is not None:
             td.decode_varlen(q, k, v, inp["seqlens"], seqlens_host=inp["seqlens_host"],
                              slopes=inp["slopes"], n_split=n_split, out=out, lse=lse,
                              stream=stream)
@@ -307,7 +341,7 @@ def run_ours(args):
 
     # end to end through the host-buffer entry point (pinned host inputs)
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and not gqa:
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
@@ -347,7 +381,8 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
                 "traffic": profiled_traffic(args.workload),
-                "kernel": "td_partial_kernel (fused ticket combine)",
+                "kernel": ("td_gqa_kernel (tcgen05)" if gqa
+                           else "td_partial_kernel (fused ticket combine)"),
                 "algorithmic_bytes_per_launch": int(bytes_step)}
 
     cpu = None
@@ -367,7 +402,7 @@ def run_ours(args):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
             "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
-                       "B": B, "H": H, "D": D, "N": N,
+                       "B": B, "H": H, "kv_heads": w.kv_heads or H, "D": D, "N": N,
                        "ragged": w.ragged is not None, "alibi": w.alibi,
                        "n_split": n_split if n_split else "auto", "parts": parts,
                        "bytes_per_step": int(bytes_step),

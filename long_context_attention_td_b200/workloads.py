@@ -43,6 +43,7 @@ class Workload:
     scale: float = 1.0
     spikes: int = 0
     seed: int = 1234
+    kv_heads: int = 0           # grouped-query: key/value heads (0 = H, plain multi-head)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -68,6 +69,12 @@ WORKLOADS = {
     # fp16 batched decode, ragged lengths U[1024, 65536], padded to 65536
     "f16_ragged_b64_h16_d64": Workload("f16_ragged_b64_h16_d64", torch.float16, 64, 16, 64,
                                        65536, ragged=(1024, 65536), seed=1238),
+    # grouped-query decode (tensor cores): 32 query heads over 8 kv heads, 128K keys
+    "gqa_bf16_h32_kv8_d128_n128k": Workload("gqa_bf16_h32_kv8_d128_n128k", torch.bfloat16, 1,
+                                            32, 128, 131072, seed=1239, kv_heads=8),
+    # multi-query decode: 32 query heads over one kv head, 1M keys
+    "mqa_bf16_h32_kv1_d128_n1m": Workload("mqa_bf16_h32_kv1_d128_n1m", torch.bfloat16, 1, 32,
+                                          128, 1 << 20, seed=1240, kv_heads=1),
 }
 
 
@@ -120,6 +127,8 @@ def make_gqa_inputs(w: Workload, Hkv: int, device="cpu"):
 
 def make_inputs(w: Workload, device="cpu"):
     """Materialise a workload: dict(q, k, v, slopes, seqlens, seqlens_host)."""
+    if w.kv_heads and w.kv_heads != w.H:
+        return make_gqa_inputs(w, w.kv_heads, device)
     device = torch.device(device)
     g = torch.Generator(device=device).manual_seed(w.seed)
     B, H, D, N = w.B, w.H, w.D, w.N
@@ -145,10 +154,11 @@ def make_inputs(w: Workload, device="cpu"):
 
 
 def kv_lengths(w: Workload, seqlens_host: Optional[torch.Tensor]) -> int:
-    """Sum over (b,h) of the keys actually attended."""
+    """Sum over (b, kv head) of the keys actually read."""
+    heads = w.kv_heads or w.H
     if seqlens_host is None:
-        return w.B * w.H * w.N
-    return int(seqlens_host.to(torch.int64).sum()) * w.H
+        return w.B * heads * w.N
+    return int(seqlens_host.to(torch.int64).sum()) * heads
 
 
 def kv_bytes(w: Workload, seqlens_host: Optional[torch.Tensor]) -> int:
