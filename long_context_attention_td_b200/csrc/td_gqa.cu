@@ -84,6 +84,19 @@ __device__ __forceinline__ void fence_before() {
 __device__ __forceinline__ void fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
+// non-blocking test of the phase with the given parity
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -835,28 +848,65 @@ __global__ void __launch_bounds__(kGqaThreads, 1)
                     const long long nt = (j1 - j0 + kTK - 1) / kTK;
                     wait(&q_ready, static_cast<uint32_t>(pc & 1));
                     fence_after();
-                    issue_S(t);
-                    if (nt > 1) issue_S(t + 1);
-                    for (long long i = 0; i < nt; ++i, ++t) {
-                        wait(&p_full[t & 1], static_cast<uint32_t>((t >> 1) & 1));
-                        fence_after();
-                        const int stage = static_cast<int>(t % kGqaStages);
-                        const uint32_t vb = sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtomBytes;
-                        const uint32_t pb = sP + static_cast<uint32_t>((t & 1) * C::kPBytes);
-                        const uint32_t dO = tmem + 128 + static_cast<uint32_t>((t & 1) * 128);
-#pragma unroll
-                        for (int kk = 0; kk < kTK / 16; ++kk) {
-                            const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
-                            const uint64_t b =
-                                smem_desc_sw128(vb + kk * 2048, C::kKVAtomBytes, 1024);
-                            // each group's first tile of the piece starts its accumulator
-                            umma_f16(dO, a, b, idO, (i > 1 || kk > 0) ? 1u : 0u);
+                    // Event loop over this piece's tiles: S products are issued in
+                    // order as soon as their K tile has landed and their S buffer is
+                    // free; P V products in order as soon as their P is written.  The
+                    // two streams interleave, so neither softmax group waits for the
+                    // other's P before its next S is issued.
+                    const long long t_end = t + nt;
+                    long long ts = t;   // next S to issue
+                    long long tp = t;   // next P V to issue
+                    uint64_t t_stall = 0;   // when the current stall began (0: none)
+                    uint32_t spins = 0;
+                    while (tp < t_end && !aborted) {
+                        bool progressed = false;
+                        if (ts < t_end &&
+                            mbar_test(smem_addr(&kv_full[ts % kGqaStages]),
+                                      static_cast<uint32_t>((ts / kGqaStages) & 1)) &&
+                            (ts < 2 || mbar_test(smem_addr(&s_empty[ts & 1]),
+                                                 static_cast<uint32_t>(((ts >> 1) - 1) & 1)))) {
+                            issue_S(ts);
+                            ++ts;
+                            progressed = true;
                         }
-                        umma_commit(smem_addr(&pv_done[t & 1]));
-                        umma_commit(smem_addr(&kv_empty[stage]));
-                        last_pv = t;
-                        if (i + 2 < nt) issue_S(t + 2);
+                        if (tp < ts && mbar_test(smem_addr(&p_full[tp & 1]),
+                                                 static_cast<uint32_t>((tp >> 1) & 1))) {
+                            fence_after();
+                            const long long i = tp - t;
+                            const int stage = static_cast<int>(tp % kGqaStages);
+                            const uint32_t vb =
+                                sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtomBytes;
+                            const uint32_t pb = sP + static_cast<uint32_t>((tp & 1) * C::kPBytes);
+                            const uint32_t dO = tmem + 128 + static_cast<uint32_t>((tp & 1) * 128);
+#pragma unroll
+                            for (int kk = 0; kk < kTK / 16; ++kk) {
+                                const uint64_t a = smem_desc_sw128(pb + kk * 32, 16, 1024);
+                                const uint64_t b =
+                                    smem_desc_sw128(vb + kk * 2048, C::kKVAtomBytes, 1024);
+                                // each group's first tile of the piece starts its accumulator
+                                umma_f16(dO, a, b, idO, (i > 1 || kk > 0) ? 1u : 0u);
+                            }
+                            umma_commit(smem_addr(&pv_done[tp & 1]));
+                            umma_commit(smem_addr(&kv_empty[stage]));
+                            last_pv = tp;
+                            ++tp;
+                            progressed = true;
+                        }
+                        if (progressed) {
+                            spins = 0;
+                            t_stall = 0;
+                        } else if ((++spins & 255u) == 0u) {
+                            const uint64_t now = global_timer_ns();
+                            if (t_stall == 0) t_stall = now;
+                            if (*abort_flag) aborted = true;
+                            else if (now - t_stall > kWaitLimitNs) {
+                                atomicOr(p.err, TD_DEVERR_WAIT_TIMEOUT);
+                                *abort_flag = 1;
+                                aborted = true;
+                            }
+                        }
                     }
+                    t = t_end;
                     ++pc;
                 } while (gwalk_next(p, ctl, w));
             }
