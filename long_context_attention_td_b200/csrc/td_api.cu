@@ -371,14 +371,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 2-D map over [rows, D] elements, box {64 columns, 64 rows}, 128-byte swizzle,
-// out-of-range rows read as zero.
-td_status make_kv_map(CUtensorMap* map, const void* base, long long rows, int D, int dtype) {
+// 2-D map over [rows, D] elements, box {64 columns, box_rows rows}, 128-byte
+// swizzle, out-of-range rows read as zero.
+td_status make_kv_map(CUtensorMap* map, const void* base, long long rows, int D, int dtype,
+                      int box_rows) {
     PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
     if (!enc) return TD_ERR_CUDA;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-    cuuint32_t box[2] = {64, 64};
+    cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
     cuuint32_t estr[2] = {1, 1};
     const CUresult rc = enc(map,
                             dtype == TD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -400,10 +401,14 @@ td_status gqa_impl(const GqaReq& r) {
     if (!mul_fits(P + 1, BHkv * r.N)) return TD_ERR_INVALID_ARG;
     const int G = r.Hq / r.Hkv;
     const size_t need = gqa_ws_bytes_for(BHkv, G, r.D, P);
+    // keys on the MMA M axis (128-key tiles) where that kernel applies, else
+    // query heads on M (64-key tiles)
+    const bool keys_path = td::gqa_keys_path(r.D, G);
+    const int box_rows = keys_path ? 128 : 64;
     CUtensorMap mk, mv;
-    st = make_kv_map(&mk, r.k, BHkv * r.N, r.D, r.dtype);
+    st = make_kv_map(&mk, r.k, BHkv * r.N, r.D, r.dtype, box_rows);
     if (st != TD_OK) return st;
-    st = make_kv_map(&mv, r.v, BHkv * r.N, r.D, r.dtype);
+    st = make_kv_map(&mv, r.v, BHkv * r.N, r.D, r.dtype, box_rows);
     if (st != TD_OK) return st;
     char* base = nullptr;
     st = prepare_ws(dev, r.ws, r.ws_bytes, BHkv, need, r.stream, &base);
@@ -432,7 +437,8 @@ td_status gqa_impl(const GqaReq& r) {
     // second kernel spreads the merge over one CTA per (sequence, query head).
     const long long per_seg = (P + BHkv - 1) / BHkv + 1;  // parts touching a sequence
     p.fused_merge = per_seg * G < kGqaSeparateMerge ? 1 : 0;
-    st = cuda_status(td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
+    st = cuda_status(keys_path ? td::launch_gqa_keys(dev, r.dtype, p, mk, mv, r.stream)
+                               : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
     if (st != TD_OK || p.fused_merge) return st;
     return cuda_status(td::launch_gqa_combine(r.D, p, r.stream));
 }
