@@ -271,7 +271,11 @@ td_status decode_impl(const Req& r) {
 
 constexpr int kGqaCtasPerSm = 1;
 // parts-per-sequence x group size above which the merge runs as its own kernel
+// (the last CTA of a sequence merges its query heads one after another; the
+// combine kernel spreads them over the SMs, worth its launch much earlier for
+// the keys-on-M kernel, whose main loop ends sooner)
 constexpr long long kGqaSeparateMerge = 128;
+constexpr long long kGqaKeysSeparateMerge = 16;
 
 // [error word][tickets][segment descriptors: 3 int32 each][part records]
 size_t gqa_desc_region(long long BHkv) { return align_up(static_cast<size_t>(BHkv) * 12, 256); }
@@ -436,7 +440,7 @@ td_status gqa_impl(const GqaReq& r) {
     // job; when many CTAs share a sequence and many query heads share it, a
     // second kernel spreads the merge over one CTA per (sequence, query head).
     const long long per_seg = (P + BHkv - 1) / BHkv + 1;  // parts touching a sequence
-    p.fused_merge = per_seg * G < kGqaSeparateMerge ? 1 : 0;
+    p.fused_merge = per_seg * G < (keys_path ? kGqaKeysSeparateMerge : kGqaSeparateMerge) ? 1 : 0;
     st = cuda_status(keys_path ? td::launch_gqa_keys(dev, r.dtype, p, mk, mv, r.stream)
                                : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
     if (st != TD_OK || p.fused_merge) return st;

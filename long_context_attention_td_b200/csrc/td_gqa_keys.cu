@@ -27,7 +27,7 @@
 //               MMAs from one lane, signalling completion with tcgen05.commit;
 //   warps 2-5   softmax group 0 (even tiles), warps 6-9 group 1 (odd tiles);
 //               warp w reads TMEM lanes 32 (w % 4) .. + 31.
-// Used for D = 128 and G <= 16; td_gqa covers the other shapes.
+// Used for D = 128 and G <= 32; td_gqa covers the other shapes.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -134,10 +134,6 @@ __device__ __forceinline__ void tmem_st_x<16>(uint32_t taddr, const uint32_t (&r
         "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
-template <>
-__device__ __forceinline__ void tmem_st_x<32>(uint32_t taddr, const uint32_t (&r)[32]) {
-    tmem_st32(taddr, r);
-}
 
 // bar.red.or over `threads` threads of named barrier `id`: true when any
 // participating thread passed true.
@@ -154,20 +150,30 @@ __device__ __forceinline__ bool bar_any(int id, int threads, bool pred) {
     return r != 0;
 }
 
-// p rounded to the element type of the P V product; returns the rounded value
+// p rounded to the element type of the P V product
 template <typename E>
-__device__ __forceinline__ float round_store(float e, unsigned char* dst);
+__device__ __forceinline__ void round_store(float e, unsigned char* dst);
 template <>
-__device__ __forceinline__ float round_store<__nv_bfloat16>(float e, unsigned char* dst) {
-    const __nv_bfloat16 r = __float2bfloat16_rn(e);
-    *reinterpret_cast<__nv_bfloat16*>(dst) = r;
-    return __bfloat162float(r);
+__device__ __forceinline__ void round_store<__nv_bfloat16>(float e, unsigned char* dst) {
+    *reinterpret_cast<__nv_bfloat16*>(dst) = __float2bfloat16_rn(e);
 }
 template <>
-__device__ __forceinline__ float round_store<__half>(float e, unsigned char* dst) {
-    const __half r = __float2half_rn(e);
-    *reinterpret_cast<__half*>(dst) = r;
-    return __half2float(r);
+__device__ __forceinline__ void round_store<__half>(float e, unsigned char* dst) {
+    *reinterpret_cast<__half*>(dst) = __float2half_rn(e);
+}
+
+// mbarrier phase test that may suspend the thread for up to `ns` nanoseconds
+// while the phase is incomplete (frees issue slots of a polling thread)
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
 }
 
 struct KCtx {
@@ -186,21 +192,26 @@ struct KCtx {
 
 // ------------------------------------------------------------ softmax role
 
-template <typename E, int GP>
+// The softmax warpgroups.  kSplit == false: group g takes the tiles with
+// t % 2 == g and every head, with its own O^T accumulator; kSplit == true:
+// both groups take every tile, group g the heads [g HG, (g+1) HG), and they
+// share one O^T accumulator (its columns are disjoint by head).
+template <typename E, int GP, bool kSplit>
 __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) {
     using C = KCfg<GP>;
     constexpr int NQ = C::NQ;
     constexpr int D = kKD;
+    constexpr int HG = kSplit ? GP / 2 : GP;    // heads of one group
     const int G = p.G;
-    const int grp = (x.warp - 2) >> 2;          // 0: even tiles, 1: odd tiles
+    const int grp = (x.warp - 2) >> 2;
+    const int hb = kSplit ? grp * HG : 0;       // first head of this group
     const int quarter = x.warp & 3;             // TMEM lane quarter of this warp
     const int lane = x.lane;
     const int key = quarter * 32 + lane;        // key of the tile (S^T row); D row of O^T
     const int st = (x.tid - 64) & (kKGroup - 1);  // thread within the group
     const int bar_grp = grp == 0 ? kBarG0 : kBarG1;
     const uint32_t lane_addr = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t s_col = static_cast<uint32_t>(grp * NQ);
-    const uint32_t o_col = static_cast<uint32_t>(2 * NQ + grp * NQ);
+    const uint32_t o_col = static_cast<uint32_t>(2 * NQ + (kSplit ? hb : grp * NQ));
     const float qscale2 = p.qscale2;
     unsigned char* smem = x.smem;
     float* stats_all = reinterpret_cast<float*>(smem + C::kOffStats);
@@ -214,6 +225,10 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                                            TD_DEVERR_WAIT_TIMEOUT))
             aborted = true;
     };
+    // wait for the P V product of tile tt (tt >= 0)
+    auto wait_pv = [&](long long tt) {
+        wait(&x.pv_done[tt & 1], static_cast<uint32_t>((tt >> 1) & 1));
+    };
     GWalk w;
     if (!gwalk_first(p, *x.ctl, w)) return;
     do {
@@ -225,8 +240,8 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         const long long qrow0 = static_cast<long long>(w.b) * p.Hq +
                                 static_cast<long long>(w.h) * G;   // first query row
         float* stats = stats_all + (pc & 1) * (2 * 4 * GP * 2 + 2 * GP);
-        float* st_l = stats;                      // [grp][quarter][h][2]
-        float* st_m = stats + 2 * 4 * GP * 2;     // [grp][h]
+        float* st_l = stats;                      // [grp][quarter][head][2]
+        float* st_m = stats + 2 * 4 * GP * 2;     // [grp][head]
 
         // Q rows of this kv head's group, K-major SW128 (rows >= G stay zero)
         if (grp == 0) {
@@ -246,33 +261,42 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
 
         float* slope2 = reinterpret_cast<float*>(smem + C::kOffSlopes) + grp * GP;
         if (p.slopes) {
-            if (st < GP) slope2[st] = st < G ? __ldg(p.slopes + w.h * G + st) * kLog2e : 0.f;
+            if (st < HG)
+                slope2[st] = hb + st < G ? __ldg(p.slopes + w.h * G + hb + st) * kLog2e : 0.f;
             named_bar_sync(bar_grp, kKGroup);
         }
-        // per head: running max (uniform in the group) and this thread's sums
-        // of p over its keys, rounded as in P (l) and unrounded (lx)
-        float m_ref[GP], l[GP], lx[GP];
+        // per head: running max m (uniform in the group; moved when a score
+        // exceeds thr = m + 8) and this thread's sum of p over its keys.  Heads
+        // past G (padding of the MMA's N) keep m = 0 and thr = +inf: their
+        // scores are 0 (zero Q rows), their p finite and never read.
+        float m_ref[HG], thr[HG], lx[HG];
 #pragma unroll
-        for (int h = 0; h < GP; ++h) {
-            m_ref[h] = kNegInf;
-            l[h] = 0.f;
+        for (int h = 0; h < HG; ++h) {
+            const bool real = hb + h < G;
+            m_ref[h] = real ? kNegInf : 0.f;
+            thr[h] = real ? kNegInf : -kNegInf;
             lx[h] = 0.f;
         }
+        // this thread's P^T element of head h: row hb + h, K column = key; with
+        // hb a multiple of HG (a power of two), (hb + h) % 8 == (hb % 8) ^ (h % 8)
+        const int kc2 = ((key & 63) >> 3) ^ (hb & 7);
+        const int p_off = (key >> 6) * C::kPAtom + (key & 7) * 2 + hb * 128;
         long long last_own = -1;
         for (long long i = 0; i < nt; ++i, ++t) {
-            if (static_cast<int>(t & 1) != grp) continue;
+            if (!kSplit && static_cast<int>(t & 1) != grp) continue;
             const long long t0 = j0 + i * kKT;
             const int rows = static_cast<int>((j1 - t0) < kKT ? (j1 - t0) : kKT);
-            wait(&x.s_full[grp], static_cast<uint32_t>((t >> 1) & 1));
+            const int buf = static_cast<int>(t & 1);
+            wait(&x.s_full[buf], static_cast<uint32_t>((t >> 1) & 1));
             fence_after();
-            uint32_t sr[GP];
-            tmem_ld_x<GP>(x.tmem + lane_addr + s_col, sr);
+            uint32_t sr[HG];
+            tmem_ld_x<HG>(x.tmem + lane_addr + static_cast<uint32_t>(buf * NQ + hb), sr);
             tmem_wait_ld();
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[grp]));
+            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[buf]));
 
-            if (rows < kKT) {
+            if (rows < kKT && (!kSplit || grp == 0)) {
                 // keys past the piece end: p is 0 there, and 0 * NaN would poison
                 // O^T, so zero those V rows before the P V product reads them
                 const int stg = static_cast<int>(t % kKStages);
@@ -288,24 +312,30 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                 fence_proxy_async_smem();
             }
 
-            // scores in log2 units; keys past the piece end and padding heads
-            // are -inf
-            const bool kvalid = key < rows;
-            const float jpos = static_cast<float>(t0 + key - w.len + 1);
-            float s[GP];
+            // scores in log2 units; keys past the piece end are -inf (the
+            // select also drops whatever those K rows hold)
+            float s[HG];
             bool need = false;
+            auto scores = [&](bool masked) {
+                const bool kvalid = key < rows;
+                const float jpos = static_cast<float>(t0 + key - w.len + 1);
 #pragma unroll
-            for (int h = 0; h < GP; ++h) {
-                const float raw = __uint_as_float(sr[h]);
-                float v = p.slopes ? fmaf(raw, qscale2, slope2[h] * jpos) : raw * qscale2;
-                v = (kvalid && h < G) ? v : kNegInf;
-                s[h] = v;
-                need |= v > m_ref[h] + kKRescale;   // m_ref = -inf: any finite score
-            }
+                for (int h = 0; h < HG; ++h) {
+                    const float raw = __uint_as_float(sr[h]);
+                    float v = p.slopes ? fmaf(raw, qscale2, slope2[h] * jpos) : raw * qscale2;
+                    if (masked) v = kvalid ? v : kNegInf;
+                    s[h] = v;
+                    need |= v > thr[h];
+                }
+            };
+            if (rows == kKT)
+                scores(false);
+            else
+                scores(true);
             if (bar_any(bar_grp, kKGroup, need)) {
                 // move the group's max to the tile max of every head
 #pragma unroll
-                for (int h = 0; h < GP; ++h) {
+                for (int h = 0; h < HG; ++h) {
                     float mx = s[h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1)
@@ -313,86 +343,100 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                     if (lane == 0) red[quarter * GP + h] = mx;
                 }
                 named_bar_sync(bar_grp, kKGroup);
-                float f[GP];
+                // O^T holds earlier tiles of the piece once a P V product of this
+                // group's columns was issued: tile t - 2 (own tiles alternate) or
+                // t - 1 (every tile)
+                const long long prev = kSplit ? (i > 0 ? t - 1 : -1) : last_own;
+                uint32_t o[HG];
+                if (prev >= 0) {
+                    wait_pv(prev);
+                    fence_after();
+                    tmem_ld_x<HG>(x.tmem + lane_addr + o_col, o);
+                    tmem_wait_ld();
+                }
 #pragma unroll
-                for (int h = 0; h < GP; ++h) {
+                for (int h = 0; h < HG; ++h) {
                     const float tm = fmaxf(fmaxf(red[h], red[GP + h]),
                                            fmaxf(red[2 * GP + h], red[3 * GP + h]));
                     const float mn = fmaxf(m_ref[h], tm);
-                    f[h] = rescale(m_ref[h], mn);
-                    m_ref[h] = mn;
-                    l[h] *= f[h];
-                    lx[h] *= f[h];
+                    const float f = rescale(m_ref[h], mn);
+                    if (hb + h < G) {
+                        m_ref[h] = mn;
+                        thr[h] = mn + kKRescale;
+                        lx[h] *= f;
+                        if (prev >= 0) o[h] = __float_as_uint(__uint_as_float(o[h]) * f);
+                    }
                 }
-                if (last_own >= 0) {
-                    // O^T holds this group's earlier tiles of the piece
-                    wait(&x.pv_done[grp], static_cast<uint32_t>(((t >> 1) - 1) & 1));
-                    fence_after();
-                    uint32_t o[GP];
-                    tmem_ld_x<GP>(x.tmem + lane_addr + o_col, o);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < GP; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * f[h]);
-                    tmem_st_x<GP>(x.tmem + lane_addr + o_col, o);
+                if (prev >= 0) {
+                    tmem_st_x<HG>(x.tmem + lane_addr + o_col, o);
                     tmem_wait_st();
                 }
                 // the maxima are read before any thread of the group can pass
                 // the next tile's reduction and overwrite them
             }
-            // the group's previous P V product (tile t - 2) read this P^T buffer
-            if (t >= 2) wait(&x.pv_done[grp], static_cast<uint32_t>(((t >> 1) - 1) & 1));
+            // the P V product of tile t - 2 read this P^T buffer
+            if (t >= 2) wait_pv(t - 2);
             fence_after();
-            unsigned char* pb =
-                smem + C::kOffP + grp * C::kPBytes + (key >> 6) * C::kPAtom + (key & 7) * 2;
-            const int kc = (key & 63) >> 3;
+            unsigned char* pb = smem + C::kOffP + buf * C::kPBytes + p_off;
 #pragma unroll
-            for (int h = 0; h < GP; ++h) {
-                if (h < G) {
-                    // masked keys give 0, also while a head has no finite max yet
-                    const float ev = s[h] == kNegInf ? 0.f : ex2(s[h] - m_ref[h]);
-                    l[h] += round_store<E>(ev, pb + swz(h, kc));
-                    lx[h] += ev;
-                }
+            for (int h = 0; h < HG; ++h) {
+                // masked keys give ex2(-inf) = 0
+                const float ev = ex2(s[h] - m_ref[h]);
+                round_store<E>(ev, pb + h * 128 + ((kc2 ^ (h & 7)) << 4));
+                lx[h] += ev;
             }
             fence_proxy_async_smem();
             fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&x.p_full[grp]));
+            if (lane == 0) mbar_arrive(smem_addr(&x.p_full[buf]));
             last_own = t;
         }
 
-        // ---- end of piece: the group's last P V product must be complete
+        // ---- end of piece: the last P V product into this group's O^T columns
+        // must be complete
         if (last_own >= 0) {
-            wait(&x.pv_done[grp], static_cast<uint32_t>((last_own >> 1) & 1));
+            wait_pv(last_own);
             fence_after();
         }
         // the group's sums per head: warp sums, then one partial per warp
+        float* my_l = st_l + (grp * 4 + quarter) * GP * 2;
 #pragma unroll
-        for (int h = 0; h < GP; ++h) {
-            if (h < G) {
-                float a = l[h], b = lx[h];
+        for (int u = 0; u < HG; ++u) {
+            // p is normalised by its unrounded sum (l = lx): sum_k r_k v_k /
+            // sum_k p_k differs from the exact average by at most the relative
+            // rounding of r times max |v|, as the rounded sum would
+            float b = 0.f;
+            if (hb + u < G) {
+                b = lx[u];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) {
-                    a += __shfl_xor_sync(0xffffffffu, a, o);
-                    b += __shfl_xor_sync(0xffffffffu, b, o);
-                }
+                for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
+            }
+            if (lane == 0) {
+                my_l[(hb + u) * 2 + 0] = b;
+                my_l[(hb + u) * 2 + 1] = b;
+            }
+            if (st == 0) st_m[grp * GP + hb + u] = m_ref[u];
+        }
+        if (kSplit) {
+            // the other group's heads: nothing from this group
+            const int ob = grp == 0 ? HG : 0;
+#pragma unroll
+            for (int u = 0; u < HG; ++u) {
                 if (lane == 0) {
-                    st_l[((grp * 4 + quarter) * GP + h) * 2 + 0] = a;
-                    st_l[((grp * 4 + quarter) * GP + h) * 2 + 1] = b;
+                    my_l[(ob + u) * 2 + 0] = 0.f;
+                    my_l[(ob + u) * 2 + 1] = 0.f;
                 }
+                if (st == 0) st_m[grp * GP + ob + u] = kNegInf;
             }
         }
-        if (st == 0)
-#pragma unroll
-            for (int h = 0; h < GP; ++h) st_m[grp * GP + h] = m_ref[h];
         fence_before();
         named_bar_sync(kBarBoth, 2 * kKGroup);
         if (grp == 0) {
             fence_after();
             // a group's O^T is stale when it had no tile of this piece
             const long long t_first = t - nt;
-            const bool has0 = nt >= 2 || (nt == 1 && (t_first & 1) == 0);
-            const bool has1 = nt >= 2 || (nt == 1 && (t_first & 1) == 1);
+            const bool has0 = kSplit || nt >= 2 || (t_first & 1) == 0;
+            const bool has1 = !kSplit && (nt >= 2 || (t_first & 1) == 1);
             uint32_t o0[GP], o1[GP];
             if (has0) tmem_ld_x<GP>(x.tmem + lane_addr + static_cast<uint32_t>(2 * NQ), o0);
             if (has1) tmem_ld_x<GP>(x.tmem + lane_addr + static_cast<uint32_t>(3 * NQ), o1);
@@ -411,8 +455,15 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                         LX += w0 * st_l[(q * GP + h) * 2 + 1] +
                               w1 * st_l[((4 + q) * GP + h) * 2 + 1];
                     }
-                    float v = has0 ? __uint_as_float(o0[h]) * w0 : 0.f;
-                    if (has1) v = fmaf(w1, __uint_as_float(o1[h]), v);
+                    // split mode: one accumulator, already relative to the
+                    // owning group's max M
+                    float v;
+                    if (kSplit) {
+                        v = __uint_as_float(o0[h]);
+                    } else {
+                        v = has0 ? __uint_as_float(o0[h]) * w0 : 0.f;
+                        if (has1) v = fmaf(w1, __uint_as_float(o1[h]), v);
+                    }
                     const long long orow = qrow0 + h;
                     if (whole) {
                         p.out[orow * D + key] = v / L;
@@ -472,7 +523,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
 
 // ------------------------------------------------------------------ kernel
 
-template <typename E, int GP>
+template <typename E, int GP, bool kSplit>
 __global__ void __launch_bounds__(kKThreads, 1)
     td_gqa_keys_kernel(const GqaParams p, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV) {
@@ -500,8 +551,9 @@ __global__ void __launch_bounds__(kKThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&s_full[s]), 1);
-            mbar_init(smem_addr(&s_empty[s]), 4);
-            mbar_init(smem_addr(&p_full[s]), 4);
+            // one arrival per softmax warp that reads S / writes P of the tile
+            mbar_init(smem_addr(&s_empty[s]), kSplit ? 8 : 4);
+            mbar_init(smem_addr(&p_full[s]), kSplit ? 8 : 4);
             mbar_init(smem_addr(&pv_done[s]), 1);
         }
         mbar_init(smem_addr(&q_ready), 8);
@@ -645,8 +697,9 @@ __global__ void __launch_bounds__(kKThreads, 1)
                             const uint32_t vb =
                                 sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtom;
                             const uint32_t pb = sP + static_cast<uint32_t>((tp & 1) * C::kPBytes);
-                            const uint32_t dO =
-                                tmem + static_cast<uint32_t>(2 * NQ + (tp & 1) * NQ);
+                            // one O^T per group (tiles alternate), or one shared
+                            const uint32_t dO = tmem + static_cast<uint32_t>(
+                                                           2 * NQ + (kSplit ? 0 : (tp & 1) * NQ));
 #pragma unroll
                             for (int kk = 0; kk < kKT / 16; ++kk) {
                                 // 16 keys: rows 16 kk.. of the V tile; the two
@@ -655,8 +708,9 @@ __global__ void __launch_bounds__(kKThreads, 1)
                                     smem_desc_sw128(vb + kk * 2048, C::kKVAtom, 1024);
                                 const uint64_t b = smem_desc_sw128(
                                     pb + (kk >> 2) * C::kPAtom + (kk & 3) * 32, 16, 1024);
-                                // each group's first tile of the piece starts its accumulator
-                                umma_f16(dO, a, b, idO, (i > 1 || kk > 0) ? 1u : 0u);
+                                // the first tile of the piece into an accumulator starts it
+                                const bool acc = (kSplit ? i > 0 : i > 1) || kk > 0;
+                                umma_f16(dO, a, b, idO, acc ? 1u : 0u);
                             }
                             umma_commit(smem_addr(&pv_done[tp & 1]));
                             umma_commit(smem_addr(&kv_empty[stage]));
@@ -667,7 +721,17 @@ __global__ void __launch_bounds__(kKThreads, 1)
                         if (progressed) {
                             spins = 0;
                             t_stall = 0;
-                        } else if ((++spins & 255u) == 0u) {
+                            continue;
+                        }
+                        // nothing ready: sleep briefly on the barrier the next
+                        // product is most likely waiting for
+                        if (tp < ts)
+                            mbar_try_wait_ns(smem_addr(&p_full[tp & 1]),
+                                             static_cast<uint32_t>((tp >> 1) & 1), 64);
+                        else if (ts < t_end)
+                            mbar_try_wait_ns(smem_addr(&kv_full[ts % kKStages]),
+                                             static_cast<uint32_t>((ts / kKStages) & 1), 64);
+                        if ((++spins & 15u) == 0u) {
                             const uint64_t now = global_timer_ns();
                             if (t_stall == 0) t_stall = now;
                             if (*abort_flag) {
@@ -695,7 +759,7 @@ __global__ void __launch_bounds__(kKThreads, 1)
         // --------------------------------------------------------- softmax
         const KCtx kx{smem, s_full, s_empty, p_full, pv_done, &q_ready, &ctl, abort_flag,
                       tmem, T, x0, x1, P, c, warp, lane, tid};
-        keys_softmax<E, GP>(p, kx);
+        keys_softmax<E, GP, kSplit>(p, kx);
     }
 
     fence_before();
@@ -707,11 +771,11 @@ __global__ void __launch_bounds__(kKThreads, 1)
     }
 }
 
-template <typename E, int GP>
+template <typename E, int GP, bool kSplit>
 cudaError_t launch_keys_t(int device, const GqaParams& p, const CUtensorMap& mk,
                           const CUtensorMap& mv, cudaStream_t s) {
     using C = KCfg<GP>;
-    auto kern = td_gqa_keys_kernel<E, GP>;
+    auto kern = td_gqa_keys_kernel<E, GP, kSplit>;
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
     if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
@@ -727,17 +791,21 @@ cudaError_t launch_keys_t(int device, const GqaParams& p, const CUtensorMap& mk,
 template <typename E>
 cudaError_t launch_keys_g(int device, const GqaParams& p, const CUtensorMap& mk,
                           const CUtensorMap& mv, cudaStream_t s) {
-    if (p.G <= 4) return launch_keys_t<E, 4>(device, p, mk, mv, s);
-    if (p.G <= 8) return launch_keys_t<E, 8>(device, p, mk, mv, s);
-    return launch_keys_t<E, 16>(device, p, mk, mv, s);
+    // up to 8 heads a thread keeps every head and the groups alternate tiles;
+    // beyond, both groups take every tile with half the heads each
+    if (p.G <= 4) return launch_keys_t<E, 4, false>(device, p, mk, mv, s);
+    if (p.G <= 8) return launch_keys_t<E, 8, false>(device, p, mk, mv, s);
+    if (p.G <= 16) return launch_keys_t<E, 16, true>(device, p, mk, mv, s);
+    return launch_keys_t<E, 32, true>(device, p, mk, mv, s);
 }
 
 }  // namespace
 
-bool gqa_keys_path(int D, int G) { return D == kKD && G >= 1 && G <= 16; }
+bool gqa_keys_path(int D, int G) { return D == kKD && G >= 1 && G <= 32; }
 
 size_t gqa_keys_smem_bytes(int G) {
-    return G <= 4 ? KCfg<4>::kSmem : G <= 8 ? KCfg<8>::kSmem : KCfg<16>::kSmem;
+    return G <= 4 ? KCfg<4>::kSmem : G <= 8 ? KCfg<8>::kSmem : G <= 16 ? KCfg<16>::kSmem
+                                                                         : KCfg<32>::kSmem;
 }
 
 cudaError_t launch_gqa_keys(int device, int dtype, const GqaParams& p, const CUtensorMap& mk,

@@ -86,7 +86,7 @@ cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const C
 // Merge the part records of every split sequence (p.fused_merge == 0).
 cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s);
 // Grouped-query kernel with the keys on the MMA M axis (td_gqa_keys.cu): same
-// parameters and part records, for D == 128 and G <= 16; its K and V tensor
+// parameters and part records, for D == 128 and G <= 32; its K and V tensor
 // maps use boxes of {64 columns, 128 rows}.
 bool gqa_keys_path(int D, int G);
 size_t gqa_keys_smem_bytes(int G);

@@ -56,7 +56,7 @@ def run_and_check(w, Hkv, n_split=0, parts=None, lens=None):
 
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("G", [1, 4, 8, 32, 128])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 8, 12, 16, 24, 32, 48, 128])
 def test_gqa_group_sizes(dtype, D, G):
     Hkv = 2
     w = Workload("gqa", dtype, 2, G * Hkv, D, 700, seed=300 + G + D)
@@ -124,3 +124,42 @@ def test_gqa_short_pieces_leave_replica_slices_empty():
     w = Workload("gqa_tiny", torch.float16, 4, 4, 64, 5, seed=901)
     for parts in (1, 3, 20):
         run_and_check(w, 1, parts=parts)
+
+
+@pytest.mark.parametrize("G", [4, 8, 16, 32])
+def test_gqa_large_groups_alibi_ragged_parts(G):
+    w = Workload("gqa_lg", torch.bfloat16, 3, G * 2, 128, 1500, alibi=True, seed=1000 + G)
+    run_and_check(w, 2, lens=[1500, 260, 1])
+    for parts in (5, 23):
+        run_and_check(w, 2, parts=parts, lens=[1500, 260, 1])
+
+
+@pytest.mark.parametrize("G", [1, 4, 8, 16, 32])
+@pytest.mark.parametrize("direction", ["growing", "shrinking"])
+def test_gqa_running_max_moves_between_tiles(G, direction):
+    """Key norms ramp along the sequence, so the score maximum moves up by many
+    log2 units from tile to tile (or only down): the kernels must rescale the
+    O accumulators they already hold."""
+    Hkv, N, D = 2, 2000, 128
+    w = Workload("gqa_ramp", torch.bfloat16, 1, G * Hkv, D, N, seed=1100 + G)
+    inp = make_gqa_inputs(w, Hkv, DEV)
+    ramp = 1.0 + torch.arange(N, device=DEV, dtype=torch.float32) / 48.0
+    if direction == "shrinking":
+        ramp = ramp.flip(0)
+    k = (inp["k"].float() * ramp[None, None, :, None]).to(w.dtype)
+    q, v = inp["q"], inp["v"]
+    for parts in (None, 3):
+        if parts is None:
+            out, lse = td.decode_gqa(q, k, v)
+            td.check_device_error()
+        else:
+            ws = torch.zeros(td.gqa_workspace_bytes(1, G * Hkv, Hkv, D, parts), dtype=torch.uint8,
+                             device=DEV)
+            out, lse = td.decode_gqa_ws(q, k, v, ws, parts=parts)
+            td.check_device_error(ws)
+        ro, rl = oracle.full_gqa(q.cpu(), k.cpu(), v.cpu())
+        o = out.reshape(-1, D).double().cpu().numpy()
+        l = lse.reshape(-1).double().cpu().numpy()
+        err_o = float(np.abs(o - ro).max())
+        assert err_o <= 4 * UNIT[w.dtype] * float(v.abs().max()), err_o
+        assert float(np.abs(l - rl).max()) <= 1e-4 * max(1.0, float(np.abs(rl).max()))
