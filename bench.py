@@ -2,8 +2,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step is one td_decode call over the whole workload: the split-KV kernel
-with its fused ticket combine (the entire hot path, one launch).  Inputs are
+One step is one decode call over the whole workload: td_decode (the split-KV
+kernel with its fused ticket combine, one launch) for multi-head workloads, or
+td_decode_gqa (the tensor-core kernel, plus the merge kernel when sequences
+are split over many CTAs) for grouped-query ones.  Inputs are
 seeded synthetic tensors already resident in HBM; the default workload
 (bf16, B=1, H=32, D=128, N=131072) moves 2 GiB of K+V per step, far beyond the
 126 MB L2, so no flush is needed between steps.  Prints one JSON line on
@@ -35,7 +37,13 @@ DEFAULT_WORKLOAD = "bf16_h32_d128_n128k"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float16: "f16"}
-KERNEL_SOURCES = ["td_partial.cu", "td_device.cuh", "td_internal.cuh"]
+# sources whose text decides each main kernel's code (its ncu summary is valid
+# while their hash matches the one recorded in it)
+KERNEL_SOURCES = {
+    "td_partial_kernel": ["td_partial.cu", "td_device.cuh", "td_internal.cuh"],
+    "td_gqa_keys_kernel": ["td_gqa_keys.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
+    "td_gqa_kernel": ["td_gqa.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
+}
 
 
 def log(*a):
@@ -51,25 +59,28 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def kernel_source_hash():
+def kernel_source_hash(kernel="td_partial_kernel"):
     h = hashlib.sha256()
-    for s in KERNEL_SOURCES:
+    for s in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "long_context_attention_td_b200", "csrc", s), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload):
-    """DRAM bytes per launch of the split-KV kernel from the committed ncu
-    summary of this workload, or None if absent or taken on other sources."""
-    path = os.path.join(ROOT, "profiles", "td_partial_%s.md" % workload)
+def profiled_traffic(workload, kernel="td_partial_kernel"):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary of this
+    workload (profiles/<kernel without _kernel>_<workload>.md), or None if
+    absent or taken on other sources."""
+    if kernel not in KERNEL_SOURCES:
+        return None
+    path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel[: -len("_kernel")], workload))
     try:
         text = open(path).read()
     except OSError:
         return None
     m_hash = re.search(r"kernel source hash:\s*`?([0-9a-f]{16})", text)
     m_bytes = re.search(r"dram bytes per launch:\s*([0-9]+)", text)
-    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash():
+    if not m_hash or not m_bytes or m_hash.group(1) != kernel_source_hash(kernel):
         return None
     return int(m_bytes.group(1))
 
@@ -306,13 +317,16 @@ def run_ours(args):
     torch.cuda.synchronize(dev)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
+    launches0 = td.launch_count()
     ev0.record(stream)
     for _ in range(args.steps):
         step()
     ev1.record(stream)
+    launches = td.launch_count() - launches0
     torch.cuda.synchronize(dev)
     barrier()
     ms_total = ev0.elapsed_time(ev1)
+    kernel_name = td.last_kernel()
     # keep the GPU loaded until the clock sampler has seen >= 1 s of load
     while time.perf_counter() - t_load0 < 1.2:
         for _ in range(20):
@@ -321,14 +335,16 @@ def run_ours(args):
     clocks = sampler.stop()
     td.check_device_error(stream=stream)
 
-    # the dominant (only) kernel per step, timed launch by launch on its stream
+    # the dominant kernel of the step, launch by launch: the library records
+    # the events on its stream right around that kernel
     n_kt = min(args.steps, 50)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n_kt)]
-    for a, b in evs:
-        a.record(stream)
-        step()
-        b.record(stream)
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            td.set_kernel_events(a, b)
+            step()
+        td.set_kernel_events(None, None)
     torch.cuda.synchronize(dev)
     kernel_ms = sum(a.elapsed_time(b) for a, b in evs) / n_kt
 
@@ -380,9 +396,8 @@ def run_ours(args):
     achieved = bytes_step / (kernel_ms_max * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                "traffic": profiled_traffic(args.workload),
-                "kernel": ("td_gqa_kernel (tcgen05)" if gqa
-                           else "td_partial_kernel (fused ticket combine)"),
+                "traffic": profiled_traffic(args.workload, kernel_name),
+                "kernel": kernel_name,
                 "algorithmic_bytes_per_launch": int(bytes_step)}
 
     cpu = None
@@ -408,7 +423,7 @@ def run_ours(args):
                        "bytes_per_step": int(bytes_step),
                        "l2": "no flush: K+V per step %.2f GB > 126 MB L2" % (bytes_step / 1e9),
                        "parallelism": "replicas x%d" % world},
-            "gpu_launches": args.steps, "clocks": clocks, "roofline": roofline,
+            "gpu_launches": int(launches), "clocks": clocks, "roofline": roofline,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

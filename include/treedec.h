@@ -278,6 +278,32 @@ TD_API int td_last_cuda_error(void);
  * (waits for the device first). */
 TD_API void td_release_workspace(void);
 
+/*
+ * Measurement hooks (no counterpart in the method; they report what the
+ * library launched, for benchmarks and tests).
+ *
+ * td_launch_count -- number of kernels launched so far by this thread's
+ * calls: the main attention kernel of every decode call (split-KV, or
+ * grouped-query), the grouped-query merge kernel when a call runs it, and
+ * td_combine's kernel.  Copies and memsets are not counted.
+ *
+ * td_set_kernel_events -- `before` and `after` are cudaEvent_t handles
+ * (created by the caller on the device of the later calls) or both NULL.
+ * While set, every decode call of this thread records `before` on its stream
+ * immediately before launching its main attention kernel and `after`
+ * immediately after, so the events' elapsed time is that kernel's duration
+ * (the grouped-query merge kernel, when it runs, comes after `after`).
+ * Errors: TD_ERR_INVALID_ARG when exactly one is NULL; a failed record is
+ * reported by the decode call as TD_ERR_CUDA.
+ *
+ * td_last_kernel -- name of the main kernel this thread's last successful
+ * launch used ("td_partial_kernel", "td_gqa_keys_kernel", "td_gqa_kernel",
+ * "td_tree_combine_kernel"; "" before the first).  Static storage.
+ */
+TD_API uint64_t td_launch_count(void);
+TD_API td_status td_set_kernel_events(void *before, void *after);
+TD_API const char *td_last_kernel(void);
+
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 TD_API int td_version(void);
 

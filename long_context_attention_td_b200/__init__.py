@@ -94,6 +94,12 @@ def lib():
     L.td_release_workspace.argtypes = []
     L.td_version.restype = i32
     L.td_version.argtypes = []
+    L.td_launch_count.restype = ctypes.c_uint64
+    L.td_launch_count.argtypes = []
+    L.td_set_kernel_events.restype = i32
+    L.td_set_kernel_events.argtypes = [vp, vp]
+    L.td_last_kernel.restype = ctypes.c_char_p
+    L.td_last_kernel.argtypes = []
     _lib = L
     return L
 
@@ -327,3 +333,30 @@ def check_device_error(workspace=None, stream=None):
 
 def release_workspace():
     lib().td_release_workspace()
+
+
+def launch_count():
+    """Kernels launched so far by this thread's library calls."""
+    return int(lib().td_launch_count())
+
+
+def last_kernel():
+    """Name of the main kernel of this thread's last library call."""
+    return lib().td_last_kernel().decode()
+
+
+def set_kernel_events(before=None, after=None):
+    """Have later calls on this thread record the torch.cuda.Events `before` and
+    `after` on their stream around their main attention kernel (None, None:
+    stop).  Each event is recorded once here first so that it exists."""
+    if (before is None) != (after is None):
+        raise ValueError("give both events or neither")
+    if before is None:
+        _check(lib().td_set_kernel_events(None, None), "td_set_kernel_events")
+        return
+    for e in (before, after):
+        if not e.cuda_event:
+            e.record()
+    _check(lib().td_set_kernel_events(ctypes.c_void_p(before.cuda_event),
+                                      ctypes.c_void_p(after.cuda_event)),
+           "td_set_kernel_events")

@@ -17,6 +17,12 @@
 namespace {
 
 thread_local int g_last_cuda = 0;
+// kernels launched by this thread's calls; events recorded around the main
+// attention kernel when set (td_set_kernel_events); name of that kernel
+thread_local unsigned long long g_launches = 0;
+thread_local cudaEvent_t g_ev_before = nullptr;
+thread_local cudaEvent_t g_ev_after = nullptr;
+thread_local const char* g_last_kernel = "";
 std::mutex g_mu;
 
 struct DevState {
@@ -66,6 +72,30 @@ void remember_workspace(const void* ws, long long tickets) {
         e->ws = ws;
     }
     e->tickets = tickets;
+}
+
+// Launch the main attention kernel of a call through `launch`, counting it and
+// recording the timing events around it when they are set.
+template <class F>
+cudaError_t launch_main(cudaStream_t s, const char* name, F&& launch) {
+    if (g_ev_before) {
+        const cudaError_t e = cudaEventRecord(g_ev_before, s);
+        if (e != cudaSuccess) return e;
+    }
+    const cudaError_t e = launch();
+    if (e != cudaSuccess) return e;
+    ++g_launches;
+    g_last_kernel = name;
+    if (g_ev_after) return cudaEventRecord(g_ev_after, s);
+    return cudaSuccess;
+}
+
+// Launch a secondary (merge) kernel through `launch`, counting it.
+template <class F>
+cudaError_t launch_aux(F&& launch) {
+    const cudaError_t e = launch();
+    if (e == cudaSuccess) ++g_launches;
+    return e;
 }
 
 td_status cuda_status(cudaError_t e) {
@@ -264,7 +294,9 @@ td_status decode_impl(const Req& r) {
     p.err = reinterpret_cast<int*>(base);
     p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
     p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BH));
-    return cuda_status(td::launch_partial(dev, r.dtype, r.D, p, r.stream));
+    return cuda_status(launch_main(r.stream, "td_partial_kernel", [&] {
+        return td::launch_partial(dev, r.dtype, r.D, p, r.stream);
+    }));
 }
 
 // ------------------------------------------------------------- grouped-query
@@ -441,10 +473,16 @@ td_status gqa_impl(const GqaReq& r) {
     // second kernel spreads the merge over one CTA per (sequence, query head).
     const long long per_seg = (P + BHkv - 1) / BHkv + 1;  // parts touching a sequence
     p.fused_merge = per_seg * G < (keys_path ? kGqaKeysSeparateMerge : kGqaSeparateMerge) ? 1 : 0;
-    st = cuda_status(keys_path ? td::launch_gqa_keys(dev, r.dtype, p, mk, mv, r.stream)
-                               : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv, r.stream));
+    st = cuda_status(launch_main(r.stream, keys_path ? "td_gqa_keys_kernel" : "td_gqa_kernel",
+                                 [&] {
+                                     return keys_path
+                                                ? td::launch_gqa_keys(dev, r.dtype, p, mk, mv,
+                                                                      r.stream)
+                                                : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv,
+                                                                 r.stream);
+                                 }));
     if (st != TD_OK || p.fused_merge) return st;
-    return cuda_status(td::launch_gqa_combine(r.D, p, r.stream));
+    return cuda_status(launch_aux([&] { return td::launch_gqa_combine(r.D, p, r.stream); }));
 }
 
 }  // namespace
@@ -547,8 +585,10 @@ td_status td_combine(const float* num, const float* m, const float* l, float* ou
     if (!aligned(num, 4) || !aligned(m, 4) || !aligned(l, 4) || !aligned(out, 4) ||
         (lse && !aligned(lse, 4)))
         return TD_ERR_INVALID_ARG;
-    return cuda_status(
-        td::launch_combine(num, m, l, out, lse, rows, S, D, reinterpret_cast<cudaStream_t>(stream)));
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(launch_main(s, "td_tree_combine_kernel", [&] {
+        return td::launch_combine(num, m, l, out, lse, rows, S, D, s);
+    }));
 }
 
 int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int num_sms) {
@@ -722,6 +762,17 @@ void td_release_workspace(void) {
     }
     cudaSetDevice(cur);
 }
+
+uint64_t td_launch_count(void) { return g_launches; }
+
+td_status td_set_kernel_events(void* before, void* after) {
+    if ((before == nullptr) != (after == nullptr)) return TD_ERR_INVALID_ARG;
+    g_ev_before = static_cast<cudaEvent_t>(before);
+    g_ev_after = static_cast<cudaEvent_t>(after);
+    return TD_OK;
+}
+
+const char* td_last_kernel(void) { return g_last_kernel; }
 
 int td_version(void) { return 100; }
 

@@ -685,9 +685,13 @@ cudaError_t launch_gqa_g(int device, const GqaParams& p, const CUtensorMap& mk,
 }  // namespace
 
 // One CTA per (sequence, query head) of the split sequences: the gist's
-// global max, renormalisation and sums over the sequence's part records.
-__global__ void __launch_bounds__(kSoftmaxThreads) td_gqa_combine_kernel(const GqaParams p, int D) {
+// global max, renormalisation and sums over the sequence's part records.  The
+// CTA's threads split each column's parts into lanes (tree_merge), so wider
+// CTAs serve sequences cut into many parts.
+template <int kThreads>
+__global__ void __launch_bounds__(kThreads) td_gqa_combine_kernel(const GqaParams p, int D) {
     __shared__ float scratch[kScratchFloats];
+    static_assert(kThreads <= kScratchFloats, "tree_merge scratch");
     const long long seg = blockIdx.x;
     const int g = blockIdx.y;
     const int n = p.seg_desc[seg * 3 + 1];
@@ -697,15 +701,22 @@ __global__ void __launch_bounds__(kSoftmaxThreads) td_gqa_combine_kernel(const G
     const long long b = seg / p.Hkv, h = seg % p.Hkv;
     const long long orow = b * p.Hq + h * p.G + g;
     const GSlotAcc acc{p.part, c_lo, first_slot, p.G, g, D};
-    tree_merge(acc, n, D, static_cast<int>(threadIdx.x), kSoftmaxThreads, scratch, kScratchFloats,
-               1, p.out + orow * D, p.lse ? p.lse + orow : nullptr);
+    tree_merge(acc, n, D, static_cast<int>(threadIdx.x), kThreads, scratch, kScratchFloats, 1,
+               p.out + orow * D, p.lse ? p.lse + orow : nullptr);
 }
 
 cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s) {
     const long long segs = static_cast<long long>(p.B) * p.Hkv;
     if (segs > 0x7fffffffLL || p.G > 65535) return cudaErrorInvalidValue;
     dim3 grid(static_cast<unsigned>(segs), static_cast<unsigned>(p.G));
-    td_gqa_combine_kernel<<<grid, kSoftmaxThreads, 0, s>>>(p, D);
+    // parts that touch one sequence, at most
+    const long long per_seg = (p.P + segs - 1) / segs + 1;
+    if (per_seg >= 64)
+        td_gqa_combine_kernel<1024><<<grid, 1024, 0, s>>>(p, D);
+    else if (per_seg >= 16)
+        td_gqa_combine_kernel<512><<<grid, 512, 0, s>>>(p, D);
+    else
+        td_gqa_combine_kernel<128><<<grid, 128, 0, s>>>(p, D);
     return cudaGetLastError();
 }
 

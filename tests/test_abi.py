@@ -144,3 +144,14 @@ def test_binding_rejects_host_tensors_for_device_calls():
     k = torch.zeros(1, 1, 8, 128, dtype=torch.bfloat16)
     with pytest.raises(TypeError):
         td.decode(q, k, k)
+
+
+def test_measurement_hooks_without_a_launch(L):
+    # nothing launched from this thread yet in a CPU-only process
+    if not torch.cuda.is_available():
+        assert td.launch_count() == 0
+        assert td.last_kernel() == ""
+    ev = ctypes.c_void_p(0x1234)
+    assert L.td_set_kernel_events(ev, None) == INVALID
+    assert L.td_set_kernel_events(None, ev) == INVALID
+    assert L.td_set_kernel_events(None, None) == 0

@@ -163,3 +163,35 @@ def test_gqa_running_max_moves_between_tiles(G, direction):
         err_o = float(np.abs(o - ro).max())
         assert err_o <= 4 * UNIT[w.dtype] * float(v.abs().max()), err_o
         assert float(np.abs(l - rl).max()) <= 1e-4 * max(1.0, float(np.abs(rl).max()))
+
+
+def test_launch_count_and_kernel_events():
+    """The library reports what it launched: one kernel for a multi-head call,
+    the grouped-query kernel plus the merge kernel when a long sequence is
+    split over the whole GPU, and events recorded right around the main kernel."""
+    w = Workload("hooks", torch.bfloat16, 1, 32, 128, 1 << 17, seed=1200)
+    inp = make_gqa_inputs(w, 1, DEV)
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    td.decode_gqa(q, k, v)
+    torch.cuda.synchronize()
+    n0 = td.launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    c, d = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    td.set_kernel_events(a, b)
+    c.record()
+    td.decode_gqa(q, k, v)
+    d.record()
+    td.set_kernel_events(None, None)
+    torch.cuda.synchronize()
+    td.check_device_error()
+    assert td.launch_count() - n0 == 2
+    assert td.last_kernel() == "td_gqa_keys_kernel"
+    k_ms, call_ms = a.elapsed_time(b), c.elapsed_time(d)
+    assert 0 < k_ms <= call_ms
+    kr = k[:, :1].expand(1, 32, w.N, 128).contiguous()
+    vr = v[:, :1].expand(1, 32, w.N, 128).contiguous()
+    n1 = td.launch_count()
+    td.decode(q, kr, vr)
+    td.check_device_error()
+    assert td.launch_count() - n1 == 1
+    assert td.last_kernel() == "td_partial_kernel"
