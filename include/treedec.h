@@ -187,6 +187,42 @@ TD_API td_status td_combine(const float *num, const float *m, const float *l, fl
                      int B, int H, int S, int D, td_stream stream);
 
 /*
+ * Sequence-sharded decode over several GPUs ("Tree Attention Decoding" gist,
+ * tree_attn_decode: each rank holds one chunk of the keys, computes its local
+ * partial attention, and the ranks exchange partial states to finish).  Here
+ * the exchange is ONE all-gather of a packed state per rank, done by the
+ * caller (e.g. NCCL through torch.distributed), instead of the gist's three
+ * all-reduces:
+ *   1. every rank: td_decode_shard on its keys -> its state buffer;
+ *   2. all-gather the states of the W ranks into one [W][state] buffer;
+ *   3. every rank: td_merge_shards -> out, lse of the whole sequence.
+ *
+ * td_decode_shard -- decode keys [key_offset, key_offset + N_shard) of every
+ * (b,h) sequence of N_total keys, held in k, v device [B,H,N_shard,D]; q as for
+ * td_decode.  ALiBi (alibi_slopes != NULL) uses each key's position in the
+ * full sequence: slope_h (key_offset + j - N_total + 1) for key j of the shard.
+ *   state  device fp32, B*H*(D+1) floats: the shard's normalised partial
+ *          outputs [B*H][D], then their natural-log log-sum-exps [B*H].
+ *   N_shard = 0 (a rank past the end of a short sequence, as torch.chunk can
+ *   leave) writes the empty state: outputs 0, log-sum-exps -inf; k and v may
+ *   then be NULL.
+ *   n_split, dtype, D, stream: as td_decode.  Requires 0 <= key_offset,
+ *   key_offset + N_shard <= N_total.  Errors as td_decode.
+ *
+ * td_merge_shards -- merge W gathered states (device fp32 [W][B*H*(D+1)], the
+ * layout td_decode_shard writes, in any rank order) into out [B,H,1,D] and
+ * lse [B,H,1] (may be NULL): the gist's global max, renormalisation and sums
+ * with (num, m, l) = (out_r, lse_r, 1).  Empty states contribute nothing.
+ * 1 <= D <= 512, W >= 1.
+ */
+TD_API td_status td_decode_shard(const void *q, const void *k, const void *v, float *state, int B,
+                                 int H, int64_t N_shard, int D, int64_t key_offset,
+                                 int64_t N_total, int n_split, const float *alibi_slopes,
+                                 td_dtype dtype, td_stream stream);
+TD_API td_status td_merge_shards(const float *states, int W, int B, int H, int D, float *out,
+                                 float *lse, td_stream stream);
+
+/*
  * td_auto_split -- the split heuristic: the number of parts (CTAs) for T =
  * B*H*N attended keys on a GPU with num_sms SMs: enough to fill every SM with
  * as many CTAs as fit at once, but no part smaller than 64 KiB of K+V and
@@ -298,7 +334,8 @@ TD_API void td_release_workspace(void);
  *
  * td_last_kernel -- name of the main kernel this thread's last successful
  * launch used ("td_partial_kernel", "td_gqa_keys_kernel", "td_gqa_kernel",
- * "td_tree_combine_kernel"; "" before the first).  Static storage.
+ * "td_tree_combine_kernel", "td_merge_shards_kernel", "td_empty_state_kernel";
+ * "" before the first).  Static storage.
  */
 TD_API uint64_t td_launch_count(void);
 TD_API td_status td_set_kernel_events(void *before, void *after);

@@ -94,6 +94,10 @@ def lib():
     L.td_release_workspace.argtypes = []
     L.td_version.restype = i32
     L.td_version.argtypes = []
+    L.td_decode_shard.restype = i32
+    L.td_decode_shard.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, i64, i64, i32, vp, i32, vp]
+    L.td_merge_shards.restype = i32
+    L.td_merge_shards.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
     L.td_launch_count.restype = ctypes.c_uint64
     L.td_launch_count.argtypes = []
     L.td_set_kernel_events.restype = i32
@@ -329,6 +333,52 @@ def check_device_error(workspace=None, stream=None):
     st = lib().td_check_device_error(ws, nbytes, ctypes.byref(bits), _stream(stream))
     if st != 0:
         raise TreeDecError(st, "kernel", "error bits 0x%x" % bits.value)
+
+
+def state_floats(B, H, D):
+    """fp32 floats of one shard state (td_decode_shard)."""
+    return B * H * (D + 1)
+
+
+def decode_shard(q, k, v, key_offset, n_total, *, state=None, slopes=None, n_split=0,
+                 stream=None):
+    """One rank's part of a sequence-sharded decode: keys [key_offset,
+    key_offset + N_shard) of sequences of n_total keys in k/v [B,H,N_shard,D].
+    Returns the packed state (fp32 [B*H*(D+1)]: outputs, then log-sum-exps)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev_tensor(t, n)
+    B, H, _, D = q.shape
+    Ns = int(k.shape[2])
+    if tuple(k.shape) != (B, H, Ns, D) or tuple(v.shape) != (B, H, Ns, D):
+        raise ValueError("k/v must be [B,H,N_shard,D] with q [B,H,1,D]")
+    if state is None:
+        state = torch.empty(state_floats(B, H, D), dtype=torch.float32, device=q.device)
+    _dev_tensor(state, "state", torch.float32)
+    if state.numel() < state_floats(B, H, D):
+        raise ValueError("state too small")
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    st = lib().td_decode_shard(_ptr(q), _ptr(k), _ptr(v), _ptr(state), B, H, Ns, D,
+                               int(key_offset), int(n_total), int(n_split), _ptr(slopes),
+                               DTYPE_CODE[q.dtype], _stream(stream))
+    _check(st, "td_decode_shard")
+    return state
+
+
+def merge_shards(states, B, H, D, *, out=None, lse=None, stream=None):
+    """Merge gathered shard states (fp32 [W, B*H*(D+1)]) into out [B,H,1,D],
+    lse [B,H,1]."""
+    _dev_tensor(states, "states", torch.float32)
+    W = states.numel() // state_floats(B, H, D)
+    if W < 1 or states.numel() != W * state_floats(B, H, D):
+        raise ValueError("states must hold W whole shard states")
+    if out is None:
+        out = torch.empty((B, H, 1, D), dtype=torch.float32, device=states.device)
+    if lse is None:
+        lse = torch.empty((B, H, 1), dtype=torch.float32, device=states.device)
+    st = lib().td_merge_shards(_ptr(states), W, B, H, D, _ptr(out), _ptr(lse), _stream(stream))
+    _check(st, "td_merge_shards")
+    return out, lse
 
 
 def release_workspace():

@@ -222,6 +222,7 @@ struct Req {
     void* ws;  // null = library-owned
     size_t ws_bytes;
     cudaStream_t stream;
+    long long alibi_off = 0;  // ALiBi position shift of a shard (see td_decode_shard)
 };
 
 td_status validate(const Req& r) {
@@ -294,6 +295,7 @@ td_status decode_impl(const Req& r) {
     p.err = reinterpret_cast<int*>(base);
     p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
     p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BH));
+    p.alibi_off = r.alibi_off;
     return cuda_status(launch_main(r.stream, "td_partial_kernel", [&] {
         return td::launch_partial(dev, r.dtype, r.D, p, r.stream);
     }));
@@ -573,6 +575,54 @@ td_status td_decode_ws(const void* q, const void* k, const void* v, float* out, 
           static_cast<int>(dtype), workspace, workspace_bytes,
           reinterpret_cast<cudaStream_t>(stream)};
     return decode_impl(r);
+}
+
+td_status td_decode_shard(const void* q, const void* k, const void* v, float* state, int B, int H,
+                          int64_t N_shard, int D, int64_t key_offset, int64_t N_total,
+                          int n_split, const float* alibi_slopes, td_dtype dtype,
+                          td_stream stream) {
+    if (!q || !state || n_split < 0 || (N_shard > 0 && (!k || !v))) return TD_ERR_INVALID_ARG;
+    if (B < 1 || H < 1 || D < 1 || N_shard < 0 || key_offset < 0 || N_total < 1)
+        return TD_ERR_INVALID_ARG;
+    if (key_offset > N_total || N_shard > N_total - key_offset) return TD_ERR_INVALID_ARG;
+    if (!aligned(state, 4)) return TD_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(B) * H;
+    if (!mul_fits(rows, static_cast<long long>(D) + 1)) return TD_ERR_INVALID_ARG;
+    float* out = state;
+    float* lse = state + rows * D;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (N_shard == 0) {
+        // no keys here (a rank past the end of a short sequence): the empty state
+        if (!dtype_ok(static_cast<int>(dtype))) return TD_ERR_UNSUPPORTED;
+        if (!d_ok(D)) return TD_ERR_UNSUPPORTED;
+        return cuda_status(launch_main(s, "td_empty_state_kernel", [&] {
+            return td::launch_empty_state(out, lse, rows, D, s);
+        }));
+    }
+    long long parts = 0;
+    if (n_split > 0) {
+        const long long per = n_split < N_shard ? n_split : N_shard;
+        parts = rows * per;
+    }
+    Req r{q, k, v, out, lse, B, H, N_shard, D, nullptr, nullptr, parts, alibi_slopes,
+          static_cast<int>(dtype), nullptr, 0, s};
+    // key j of the shard sits at key_offset + j of the N_total keys
+    r.alibi_off = key_offset + N_shard - N_total;
+    return decode_impl(r);
+}
+
+td_status td_merge_shards(const float* states, int W, int B, int H, int D, float* out,
+                          float* lse, td_stream stream) {
+    if (!states || !out || W < 1 || B < 1 || H < 1 || D < 1 || D > 512) return TD_ERR_INVALID_ARG;
+    const long long rows = static_cast<long long>(B) * H;
+    if (rows > 0x7fffffffLL || !mul_fits(rows * (D + 1), static_cast<long long>(W) * 4))
+        return TD_ERR_INVALID_ARG;
+    if (!aligned(states, 4) || !aligned(out, 4) || (lse && !aligned(lse, 4)))
+        return TD_ERR_INVALID_ARG;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return cuda_status(launch_main(s, "td_merge_shards_kernel", [&] {
+        return td::launch_merge_shards(states, W, rows, D, out, lse, s);
+    }));
 }
 
 td_status td_combine(const float* num, const float* m, const float* l, float* out, float* lse,

@@ -59,6 +59,8 @@ struct PartialParams {
     float* part;             // part records
     int* tickets;            // [B*H]
     int* err;                // error word
+    int64_t alibi_off;       // ALiBi position of key j is j - n + 1 + alibi_off (0: the
+                             // sequence is whole; a shard adds its place in the full one)
 };
 
 // Grouped-query kernel (td_gqa.cu): Hq = G * Hkv query heads over Hkv kv heads.
@@ -98,6 +100,12 @@ size_t partial_smem_bytes(int dtype, int D);
 // CTAs of the split-KV kernel that fit on one SM (static estimate from shared
 // memory and threads; matches the kernel's launch bounds).
 int partial_ctas_per_sm(int dtype, int D);
+// Empty partial state (out 0, lse -inf) of `rows` (b,h) rows: a shard with no keys.
+cudaError_t launch_empty_state(float* out, float* lse, long long rows, int D, cudaStream_t s);
+// Merge W gathered shard states [W][rows*D | rows] into out[rows][D], lse[rows].
+cudaError_t launch_merge_shards(const float* states, int W, long long rows, int D, float* out,
+                                float* lse, cudaStream_t s);
+
 // Launch the split-KV kernel (grid = p.P) with its fused combine on `device`
 // (the current device).
 cudaError_t launch_partial(int device, int dtype, int D, const PartialParams& p, cudaStream_t s);

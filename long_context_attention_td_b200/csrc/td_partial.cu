@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         const float qscale2 = p.qscale2;
         const bool has_bias = p.slopes != nullptr;
         const float slope2 = has_bias ? __ldg(p.slopes + w.h) * kLog2e : 0.f;
+        const long long pos0 = 1 - w.len + p.alibi_off;   // ALiBi position of key 0
 
         float m = kNegInf, l = 0.f;
         float acc[C::kNV][C::kVec];
@@ -360,7 +361,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 const int row = gi + i * C::kNG;
                 if (row < rows) {
                     s[i] = has_bias
-                               ? fmaf(s[i], qscale2, slope2 * static_cast<float>(t0 + row - w.len + 1))
+                               ? fmaf(s[i], qscale2, slope2 * static_cast<float>(t0 + row + pos0))
                                : s[i] * qscale2;
                     tmax = fmaxf(tmax, s[i]);
                 } else {

@@ -155,3 +155,17 @@ def test_measurement_hooks_without_a_launch(L):
     assert L.td_set_kernel_events(ev, None) == INVALID
     assert L.td_set_kernel_events(None, ev) == INVALID
     assert L.td_set_kernel_events(None, None) == 0
+
+
+def test_shard_entry_points_reject_bad_arguments(L):
+    p = ctypes.c_void_p(256)
+    # keys past the end of the full sequence, negative offset, empty total
+    assert L.td_decode_shard(p, p, p, p, 1, 1, 10, 128, 5, 12, 0, None, 1, None) == INVALID
+    assert L.td_decode_shard(p, p, p, p, 1, 1, 10, 128, -1, 12, 0, None, 1, None) == INVALID
+    assert L.td_decode_shard(p, p, p, p, 1, 1, 0, 128, 0, 0, 0, None, 1, None) == INVALID
+    assert L.td_decode_shard(p, None, None, None, 1, 1, 0, 128, 0, 4, 0, None, 1, None) == INVALID
+    # keys present but no k/v pointers
+    assert L.td_decode_shard(p, None, p, p, 1, 1, 3, 128, 0, 4, 0, None, 1, None) == INVALID
+    assert L.td_merge_shards(p, 0, 1, 1, 128, p, p, None) == INVALID
+    assert L.td_merge_shards(p, 2, 1, 1, 1024, p, p, None) == INVALID
+    assert L.td_merge_shards(None, 2, 1, 1, 128, p, p, None) == INVALID

@@ -6,6 +6,8 @@
    two all-reduce SUMs -- the result must equal the plain definition.
 2. bench.py's rank aggregation: max of the timed region over ranks, sum of the
    work, and one JSON line from rank 0 only.
+3. The library's sequence-sharded decode (long_context_attention_td_b200.sharded):
+   its plumbing on gloo ranks, with the oracle standing in for its two kernels.
 """
 import math
 import os
@@ -118,3 +120,101 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
     monkeypatch.setenv("RANK", "1")
     bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3"])
     assert capsys.readouterr().out == ""
+
+
+# ------------------------------------------------ sequence-sharded decode
+
+def _oracle_shard_state(q, k_s, v_s, off, n_total, slopes=None, n_split=0, stream=None):
+    """td_decode_shard's contract computed by the oracle: each (b,h) attends
+    its shard's keys with the ALiBi term of their place in the full sequence."""
+    import oracle
+    B, H, _, D = q.shape
+    ns = k_s.shape[2]
+    out = np.zeros((B * H, D))
+    lse = np.full(B * H, -np.inf)
+    for b in range(B):
+        for h in range(H):
+            if ns == 0:
+                continue
+            slope = 0.0 if slopes is None else float(slopes[h])
+            extra = np.full(ns, slope * (off + ns - n_total))
+            o, l = oracle.attend_one(q[b, h, 0], k_s[b, h], v_s[b, h], slope=slope,
+                                     extra_bias=extra)
+            out[b * H + h] = o
+            lse[b * H + h] = l
+    return torch.from_numpy(np.concatenate([out.ravel(), lse])).to(torch.float32)
+
+
+def _oracle_merge(gathered, B, H, D, stream=None):
+    import oracle
+    W = gathered.shape[0]
+    g = gathered.double().numpy()
+    outs = g[:, : B * H * D].reshape(W, B * H, D)
+    lses = g[:, B * H * D:]
+    out = np.zeros((B * H, D))
+    lse = np.zeros(B * H)
+    for row in range(B * H):
+        m = lses[:, row]
+        o, l = oracle.merge(outs[:, row], m, np.isfinite(m).astype(np.float64))
+        out[row], lse[row] = o, l
+    return out, lse
+
+
+def _sharded(rank, world, port, n, mode, alibi, result):
+    from long_context_attention_td_b200 import sharded
+    _init(rank, world, port)
+    try:
+        B, H, D = 2, 3, 32
+        g = torch.Generator().manual_seed(7 + n)
+        q = torch.randn(B, H, 1, D, generator=g)
+        k = torch.randn(B, H, n, D, generator=g)
+        v = torch.randn(B, H, n, D, generator=g)
+        slopes = torch.tensor([0.5, 0.25, 0.125]) if alibi else None
+        off, ln = sharded.shard_bounds(n, world, mode)[rank]
+        out, lse = sharded.decode_sharded(q, k[:, :, off:off + ln], v[:, :, off:off + ln], off, n,
+                                          slopes=slopes, shard_fn=_oracle_shard_state,
+                                          merge_fn=_oracle_merge)
+        result.put((rank, out.tolist(), lse.tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,n,mode,alibi", [(2, 37, "torch_chunk", True), (3, 2, "torch_chunk", False),
+                                                (3, 100, "balanced", True), (2, 1, "balanced", True)])
+def test_sharded_decode_on_cpu_ranks(world, n, mode, alibi):
+    """decode_sharded's plumbing -- chunk bounds, the packed state, the one
+    all-gather in rank order, the merge -- on gloo ranks, with the two kernels
+    replaced by the oracle computing their stated contracts; every rank must
+    end with the plain definition over the whole sequence."""
+    import oracle
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_sharded, args=(r, world, port, n, mode, alibi, result))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [result.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    B, H, D = 2, 3, 32
+    g = torch.Generator().manual_seed(7 + n)
+    q = torch.randn(B, H, 1, D, generator=g)
+    k = torch.randn(B, H, n, D, generator=g)
+    v = torch.randn(B, H, n, D, generator=g)
+    slopes = np.array([0.5, 0.25, 0.125], dtype=np.float32) if alibi else None
+    ref, ref_l = oracle.full(q, k, v, slopes=slopes)
+    for _, out, lse in got:
+        np.testing.assert_allclose(np.array(out), ref, rtol=0, atol=2e-6)
+        np.testing.assert_allclose(np.array(lse), ref_l, rtol=0, atol=2e-6)
+
+
+@pytest.mark.parametrize("n,world", [(0, 1), (1, 4), (5, 4), (31, 8), (4096, 8), (1000, 3)])
+def test_shard_bounds_match_the_oracle_chunking(n, world):
+    import oracle
+    from long_context_attention_td_b200 import sharded
+    for mode in ("torch_chunk", "balanced"):
+        starts = oracle.chunk_bounds(n, world, mode)
+        got = sharded.shard_bounds(n, world, mode)
+        assert [(a, b - a) for a, b in zip(starts[:-1], starts[1:])] == got
