@@ -432,6 +432,109 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------- sequence-sharded (strong scaling)
+
+def run_sharded(args):
+    """--shard-seq: every sequence of the workload is split over the N ranks
+    (the gist's setting: rank r holds chunk r of the keys); a step is
+    td_decode_shard on the rank's chunk, one all-gather of the packed states
+    and td_merge_shards.  The total work is fixed, so this is strong scaling."""
+    import long_context_attention_td_b200 as td
+    from long_context_attention_td_b200 import sharded
+
+    world, rank, local = dist_setup(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    if (w.kv_heads and w.kv_heads != w.H) or w.ragged is not None:
+        raise SystemExit("--shard-seq takes a uniform multi-head workload")
+    if args.n_keys:
+        w = w.with_(N=args.n_keys)
+    off, ln = sharded.shard_bounds(w.N, world, "balanced")[rank]
+    # same seed on every rank: q is the same query everywhere; the chunk's
+    # key values do not matter for timing
+    inp = make_inputs(w.with_(N=max(ln, 1)), dev)
+    q, k, v, slopes = inp["q"], inp["k"][:, :, :ln], inp["v"][:, :, :ln], inp["slopes"]
+    k, v = k.contiguous(), v.contiguous()
+    stream = torch.cuda.current_stream(dev)
+    n_split = w.n_split if args.n_split is None else args.n_split
+    B, H, D, N = w.B, w.H, w.D, w.N
+    bytes_all = float(2 * B * H * N * D * w.elt)
+
+    def step():
+        sharded.decode_sharded(q, k, v, off, N, slopes=slopes, n_split=n_split, stream=stream)
+
+    sampler = ClockSampler(dev.index).start()
+    t_load0 = time.perf_counter()
+    for _ in range(args.warmup):
+        step()
+    td.check_device_error(stream=stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches0 = td.launch_count()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    launches = td.launch_count() - launches0
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    while time.perf_counter() - t_load0 < 1.2:
+        for _ in range(20):
+            step()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    td.check_device_error(stream=stream)
+    # this rank's shard kernel alone, launch by launch
+    n_kt = min(args.steps, 50)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_kt)]
+    state = torch.empty(td.state_floats(B, H, D), dtype=torch.float32, device=dev)
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            td.set_kernel_events(a, b)
+            td.decode_shard(q, k, v, off, N, state=state, slopes=slopes, n_split=n_split,
+                            stream=stream)
+        td.set_kernel_events(None, None)
+    torch.cuda.synchronize(dev)
+    kernel_name = td.last_kernel()
+    kernel_ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / n_kt, dev)
+    ms_max = reduce_max(ms_total, dev)
+    ms_per_step = ms_max / args.steps
+    peak, peak_kind = measured_peak()
+    shard_bytes = 2 * B * H * ln * D * w.elt
+    achieved = shard_bytes / (kernel_ms * 1e-3) / 1e9 if ln else 0.0
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(bytes_all / (ms_per_step * 1e-3) / 1e9, 3),
+            "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "us_per_step": round(ms_per_step * 1e3, 3),
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
+            "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
+            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
+                       "B": B, "H": H, "D": D, "N": N, "alibi": w.alibi,
+                       "bytes_per_step": int(bytes_all),
+                       "l2": "no flush: K+V per rank per step %.2f GB > 126 MB L2" % (shard_bytes / 1e9),
+                       "parallelism": "sequence-sharded x%d" % world,
+                       "collective": "one all_gather of B*H*(D+1) fp32 per rank"},
+            "gpu_launches": int(launches), "clocks": clocks,
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": peak_kind, "traffic": None, "kernel": kernel_name,
+                         "algorithmic_bytes_per_launch": int(shard_bytes)},
+            "e2e": None, "cpu_baseline": None,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 # -------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -482,11 +585,16 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard-seq", action="store_true",
+                    help="split every sequence over the ranks (one all-gather per step) "
+                         "instead of giving each rank its own workload")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard_seq:
+        run_sharded(args)
     else:
         run_ours(args)
 

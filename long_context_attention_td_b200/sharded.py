@@ -63,12 +63,17 @@ def decode_sharded(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor
     """
     shard_fn = shard_fn or decode_shard
     merge_fn = merge_fn or merge_shards
-    world = dist.get_world_size(group)
+    # one process without a process group: a single shard, nothing to exchange
+    alone = group is None and not (dist.is_available() and dist.is_initialized())
+    world = 1 if alone else dist.get_world_size(group)
     B, H, _, D = q.shape
     state = shard_fn(q, k_shard, v_shard, key_offset, n_total, slopes=slopes, n_split=n_split,
                      stream=stream)
     if state.numel() != state_floats(B, H, D):
         raise ValueError("shard state has the wrong size")
-    gathered = torch.empty((world, state.numel()), dtype=torch.float32, device=state.device)
-    _all_gather(gathered, state, group)
+    if alone:
+        gathered = state.view(1, -1)
+    else:
+        gathered = torch.empty((world, state.numel()), dtype=torch.float32, device=state.device)
+        _all_gather(gathered, state, group)
     return merge_fn(gathered, B, H, D, stream=stream)

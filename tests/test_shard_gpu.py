@@ -70,3 +70,15 @@ def test_all_empty_states_merge_to_zero():
     td.check_device_error()
     assert torch.count_nonzero(out) == 0
     assert torch.all(torch.isinf(lse)) and torch.all(lse < 0)
+
+
+def test_decode_sharded_in_one_process():
+    """The distributed entry point without a process group: one shard holding
+    the whole sequence, merged with itself."""
+    w = Workload("shard_one", torch.float16, 1, 8, 64, 20000, alibi=True, seed=1400)
+    inp = make_inputs(w, DEV)
+    out, lse = sharded.decode_sharded(inp["q"], inp["k"], inp["v"], 0, w.N, slopes=inp["slopes"])
+    td.check_device_error()
+    ro, rl = oracle.full(inp["q"].cpu(), inp["k"].cpu(), inp["v"].cpu(), slopes=inp["slopes"].cpu())
+    assert float(np.abs(out.reshape(-1, w.D).double().cpu().numpy() - ro).max()) <= SPEC_OUT[w.dtype]
+    assert float(np.abs(lse.reshape(-1).double().cpu().numpy() - rl).max()) <= SPEC_LSE
