@@ -10,8 +10,9 @@ the GPU sees) or numpy float32/float16 arrays.  Results are numpy float64.
 Sources (page title -- section):
   "Tree Attention Decoding" gist, tree_attn_decode.py -- regular_decode and
   tree_attn_decode (Algorithm 3); llm-foundry issue #186 "ALiBi with
-  causal=True unexpected bias?" -- the broadcast bias row; "Flash Aandacht"
-  (unite.ai) -- "De Wiskunde Achter Flash Aandacht", formulas 1 and 2.
+  causal=True unexpected bias?" -- the broadcast bias row and causal masking;
+  "Flash Aandacht" (unite.ai) -- "De Wiskunde Achter Flash Aandacht", formulas
+  1 and 2, and the blockwise forward it describes (whose rows prefill computes).
 """
 import ctypes
 import os
@@ -59,6 +60,10 @@ def lib():
         L.or_full_gqa.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                   ctypes.c_int, ctypes.c_int64, ctypes.c_int, vp, vp, vp,
                                   ctypes.c_int64, vp, vp, ctypes.c_int]
+        L.or_prefill.restype = ctypes.c_int
+        L.or_prefill.argtypes = [vp, vp, vp, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                 ctypes.c_int64, ctypes.c_int, ctypes.c_int, vp, vp,
+                                 ctypes.c_int64, vp, vp, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -148,6 +153,28 @@ def full_gqa(q, k, v, slopes=None, seqlens=None, bh=None, threads=0):
     lse = np.zeros((n_bh,), dtype=np.float64)
     _check(lib().or_full_gqa(pq, pk, pv, cq, B, H, Hkv, Nmax, D, _ptr(sq), _ptr(sl), _ptr(bl),
                              n_bh, out.ctypes.data, lse.ctypes.data, int(threads)), "full_gqa")
+    return out, lse
+
+
+def prefill(q, k, v, causal=True, slopes=None, rows=None, threads=0):
+    """Prefill attention of every query row (or the listed row indices
+    (b*H + h)*S + i): q, k, v [B,H,S,D]; slope_h (j - S + 1) bias; causal mask
+    j <= i when causal.  Returns (out [n_rows, D], lse [n_rows]) in fp64."""
+    cq, tq, pq = _code_and_buf(q)
+    ck, tk, pk = _code_and_buf(k)
+    cv, tv, pv = _code_and_buf(v)
+    if not (cq == ck == cv):
+        raise TypeError("q, k, v must share one element type")
+    B, H, S, D = tuple(tq.shape)
+    if tuple(tk.shape) != (B, H, S, D) or tuple(tv.shape) != (B, H, S, D):
+        raise ValueError("layout must be q, k, v [B,H,S,D]")
+    sl = None if slopes is None else np.ascontiguousarray(np.asarray(slopes, dtype=np.float32))
+    rl = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    n = B * H * S if rl is None else len(rl)
+    out = np.zeros((n, D), dtype=np.float64)
+    lse = np.zeros((n,), dtype=np.float64)
+    _check(lib().or_prefill(pq, pk, pv, cq, B, H, S, D, 1 if causal else 0, _ptr(sl), _ptr(rl), n,
+                            out.ctypes.data, lse.ctypes.data, int(threads)), "prefill")
     return out, lse
 
 

@@ -386,6 +386,108 @@ int or_full_gqa(const void *q, const void *k, const void *v, int dtype, int B, i
     return run(&J, threads);
 }
 
+/* ---------------------------------------------------------------- prefill */
+
+/*
+ * Prefill attention of every query row of a sequence of S tokens: the plain
+ * definition with the [ALIBI] bias row over the whole sequence and, when
+ * causal, its causal mask ([ALIBI] causal=True; [FA] "Flash Aandacht"
+ * computes the same rows blockwise):
+ *   s_ij = (q_i D^-1/2) . k_j + slope_h (j - S + 1)   for j in J(i),
+ *   J(i) = {0, .., i} if causal else {0, .., S-1},
+ *   m_i = max_j s_ij, out_i = sum_j e^(s_ij - m_i) v_j / sum_j e^(s_ij - m_i),
+ *   lse_i = m_i + ln sum_j e^(s_ij - m_i).
+ * Layout q, k, v [B,H,S,D]; `rows` lists row indices (b*H + h)*S + i (all
+ * B*H*S rows when NULL); out [n_rows, D], lse [n_rows] fp64.
+ */
+typedef struct {
+    const void *q, *k, *v;
+    int dtype, B, H, D, causal;
+    int64_t S;
+    const float *slopes;
+    const int64_t *rows;
+    int64_t n_rows;
+    double *out, *lse;
+    int64_t next;
+    int rc;
+} prefill_job_t;
+
+static int prefill_row(const prefill_job_t *J, int64_t r, double *out, double *lse) {
+    const int D = J->D;
+    const int64_t S = J->S;
+    const int64_t bh = r / S, i = r % S;
+    const int64_t h = bh % J->H;
+    const double slope = J->slopes ? (double)J->slopes[h] : 0.0;
+    const int64_t nk = J->causal ? i + 1 : S;
+    const int64_t kv_off = bh * S * (int64_t)D;
+    double *s = (double *)malloc(sizeof(double) * (size_t)nk);
+    double *o = (double *)calloc((size_t)D, sizeof(double));
+    double *qs = (double *)malloc(sizeof(double) * (size_t)D);
+    if (!s || !o || !qs) {
+        free(s);
+        free(o);
+        free(qs);
+        return -2;
+    }
+    const double scale = 1.0 / sqrt((double)D);
+    for (int d = 0; d < D; ++d) qs[d] = load_elem(J->q, r * (int64_t)D + d, J->dtype) * scale;
+    double m = -INFINITY;
+    for (int64_t j = 0; j < nk; ++j) {
+        double acc = 0.0;
+        for (int d = 0; d < D; ++d) acc += qs[d] * load_elem(J->k, kv_off + j * (int64_t)D + d, J->dtype);
+        acc += or_alibi_bias(slope, j, S);
+        s[j] = acc;
+        if (acc > m) m = acc;
+    }
+    double l = 0.0;
+    for (int64_t j = 0; j < nk; ++j) {
+        const double p = exp(s[j] - m);
+        l += p;
+        for (int d = 0; d < D; ++d) o[d] += p * load_elem(J->v, kv_off + j * (int64_t)D + d, J->dtype);
+    }
+    for (int d = 0; d < D; ++d) out[d] = o[d] / l;
+    *lse = m + log(l);
+    free(s);
+    free(o);
+    free(qs);
+    return 0;
+}
+
+static void *prefill_worker(void *arg) {
+    prefill_job_t *J = (prefill_job_t *)arg;
+    for (;;) {
+        int64_t i = __atomic_fetch_add(&J->next, 1, __ATOMIC_RELAXED);
+        if (i >= J->n_rows) break;
+        int64_t r = J->rows ? J->rows[i] : i;
+        int rc = prefill_row(J, r, J->out + i * (int64_t)J->D, J->lse + i);
+        if (rc) __atomic_store_n(&J->rc, rc, __ATOMIC_RELAXED);
+    }
+    return NULL;
+}
+
+int or_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int64_t S,
+               int D, int causal, const float *slopes, const int64_t *rows, int64_t n_rows,
+               double *out, double *lse, int threads) {
+    if (!q || !k || !v || !out || !lse || dtype < OR_F32 || dtype > OR_F16 || B <= 0 ||
+        H <= 0 || S <= 0 || D <= 0 || n_rows < 0)
+        return -1;
+    prefill_job_t J = {q, k, v, dtype, B, H, D, causal ? 1 : 0, S, slopes, rows,
+                       rows ? n_rows : (int64_t)B * H * S, out, lse, 0, 0};
+    if (rows)
+        for (int64_t i = 0; i < n_rows; ++i)
+            if (rows[i] < 0 || rows[i] >= (int64_t)B * H * S) return -1;
+    if (threads <= 0) threads = (int)sysconf(_SC_NPROCESSORS_ONLN);
+    if (threads < 1) threads = 1;
+    if (threads > 256) threads = 256;
+    pthread_t tid[256];
+    int started = 0;
+    for (int t = 1; t < threads; ++t)
+        if (pthread_create(&tid[started], NULL, prefill_worker, &J) == 0) ++started;
+    prefill_worker(&J);
+    for (int t = 0; t < started; ++t) pthread_join(tid[t], NULL);
+    return J.rc;
+}
+
 /* The same, through the chunked Algorithm-3 path with w chunks per (b,h). */
 int or_chunked(const void *q, const void *k, const void *v, int dtype, int B, int H,
                int64_t Nmax, int D, const int32_t *seqlens, const float *slopes,

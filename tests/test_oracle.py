@@ -443,3 +443,109 @@ def test_gqa_vs_torch_sdpa_enable_gqa():
     ref = torch.nn.functional.scaled_dot_product_attention(
         q.double(), k.double(), v.double(), enable_gqa=True)
     np.testing.assert_allclose(o, ref.reshape(B * H, D).numpy(), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------- prefill
+
+def _prefill_block_loop_corrected(q, k, v, slope, causal, qblk, kblk):
+    """The Flash Aandacht blockwise forward (outer loop over query blocks,
+    inner over key blocks, running M, L and O per query row), with the
+    normalised O rescaled by L before it is updated, the ALiBi broadcast row
+    slope (j - S + 1) and, when causal, the mask j > i; fp64 numpy."""
+    S, D = q.shape
+    s_all = (q @ k.T) / math.sqrt(D) + slope * (np.arange(S) - S + 1)[None, :]
+    O = np.zeros((S, D))
+    L = np.zeros(S)
+    M = np.full(S, -math.inf)
+    for i0 in range(0, S, qblk):
+        rows = np.arange(i0, min(S, i0 + qblk))
+        for j0 in range(0, S, kblk):
+            cols = np.arange(j0, min(S, j0 + kblk))
+            sb = s_all[np.ix_(rows, cols)].copy()
+            if causal:
+                sb[cols[None, :] > rows[:, None]] = -math.inf
+            Mn = np.maximum(M[rows], sb.max(axis=1))
+            ok = Mn != -math.inf
+            e = np.where(ok[:, None], np.exp(sb - np.where(ok, Mn, 0.0)[:, None]), 0.0)
+            a = np.where(M[rows] != -math.inf, np.exp(M[rows] - np.where(ok, Mn, 0.0)), 0.0)
+            Ln = a * L[rows] + e.sum(axis=1)
+            O[rows] = np.where(Ln[:, None] > 0,
+                               (a[:, None] * L[rows][:, None] * O[rows] + e @ v[cols])
+                               / np.where(Ln > 0, Ln, 1.0)[:, None], 0.0)
+            L[rows], M[rows] = Ln, Mn
+    return O, M + np.log(L)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("slope", [0.0, 0.37])
+@pytest.mark.parametrize("qblk,kblk", [(1, 1), (4, 7), (16, 5), (64, 64)])
+def test_prefill_matches_the_corrected_blockwise_forward(causal, slope, qblk, kblk):
+    S, D = 37, 16
+    q = _rand((S, D), torch.float32, 181).double().numpy()
+    k = _rand((S, D), torch.float32, 182).double().numpy()
+    v = _rand((S, D), torch.float32, 183).double().numpy()
+    o, l = oracle.prefill(torch.from_numpy(q).float()[None, None], torch.from_numpy(k).float()[None, None],
+                          torch.from_numpy(v).float()[None, None], causal=causal,
+                          slopes=np.array([slope], dtype=np.float32))
+    bo, bl = _prefill_block_loop_corrected(q, k, v, np.float32(slope), causal, qblk, kblk)
+    np.testing.assert_allclose(o, bo, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(l, bl, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_prefill_vs_torch_sdpa_causal(dtype):
+    """Library pin: fp64 SDPA with the causal mask plus the ALiBi row as an
+    additive mask, on the exactly widened inputs."""
+    B, H, S, D = 2, 3, 29, 32
+    q = _rand((B, H, S, D), dtype, 191)
+    k = _rand((B, H, S, D), dtype, 192)
+    v = _rand((B, H, S, D), dtype, 193)
+    slopes = np.array([0.5, 0.0, 0.125], dtype=np.float32)
+    o, _ = oracle.prefill(q, k, v, causal=True, slopes=slopes)
+    row = torch.arange(S, dtype=torch.float64) - S + 1
+    mask = torch.full((S, S), -math.inf, dtype=torch.float64).triu(1)
+    bias = torch.from_numpy(slopes.astype(np.float64))[:, None, None] * row[None, None, :] + mask
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double(), k.double(), v.double(),
+                                                           attn_mask=bias[None])
+    np.testing.assert_allclose(o, ref.reshape(-1, D).numpy(), rtol=0, atol=1e-12)
+
+
+def test_prefill_rows_are_decodes_of_their_prefixes():
+    """Causal row i is a decode of the first i + 1 keys whose ALiBi row is
+    shifted by the constant slope (i + 1 - S): out equal, lse shifted; the last
+    row is exactly the decode of the whole sequence; non-causal rows are
+    decodes of the whole sequence."""
+    S, D, slope = 23, 8, 0.25
+    q = _rand((1, 1, S, D), torch.bfloat16, 201)
+    k = _rand((1, 1, S, D), torch.bfloat16, 202)
+    v = _rand((1, 1, S, D), torch.bfloat16, 203)
+    o, l = oracle.prefill(q, k, v, causal=True, slopes=np.array([slope], dtype=np.float32))
+    for i in range(S):
+        ro, rl = oracle.attend_one(q[0, 0, i], k[0, 0, :i + 1], v[0, 0, :i + 1], slope=slope)
+        np.testing.assert_allclose(o[i], ro, rtol=0, atol=1e-12)
+        assert abs(l[i] - (rl + slope * (i + 1 - S))) < 1e-12
+    ro, rl = oracle.attend_one(q[0, 0, S - 1], k[0, 0], v[0, 0], slope=slope)
+    np.testing.assert_array_equal(o[S - 1], ro)
+    assert l[S - 1] == rl
+    on, ln = oracle.prefill(q, k, v, causal=False, slopes=np.array([slope], dtype=np.float32))
+    for i in (0, 7, S - 1):
+        ro, rl = oracle.attend_one(q[0, 0, i], k[0, 0], v[0, 0], slope=slope)
+        np.testing.assert_allclose(on[i], ro, rtol=0, atol=1e-12)
+        assert abs(ln[i] - rl) < 1e-12
+
+
+def test_prefill_first_row_closed_form_and_row_selection():
+    S, D, slope = 9, 4, 0.5
+    q = _rand((2, 2, S, D), torch.float32, 211)
+    k = _rand((2, 2, S, D), torch.float32, 212)
+    v = _rand((2, 2, S, D), torch.float32, 213)
+    o, l = oracle.prefill(q, k, v, causal=True, slopes=np.array([slope, 0.0], dtype=np.float32))
+    # row 0 of a causal prefill sees key 0 only
+    np.testing.assert_array_equal(o[0], v[0, 0, 0].double().numpy())
+    s00 = float((q[0, 0, 0].double() * k[0, 0, 0].double()).sum()) / 2.0 + slope * (1 - S)
+    assert abs(l[0] - s00) < 1e-12
+    rows = [0, S + 3, 3 * S + 8, 2 * S]
+    os_, ls_ = oracle.prefill(q, k, v, causal=True, slopes=np.array([slope, 0.0], dtype=np.float32),
+                              rows=rows)
+    np.testing.assert_array_equal(os_, o[rows])
+    np.testing.assert_array_equal(ls_, l[rows])
