@@ -30,9 +30,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from long_context_attention_td_b200.workloads import WORKLOADS, kv_bytes, kv_lengths, make_inputs  # noqa: E402
+from long_context_attention_td_b200.workloads import (WORKLOADS, kv_bytes, kv_lengths,  # noqa: E402
+                                                      make_inputs, prefill_flops)
 
 METRIC = "decode attention KV GB/s and % of B200 HBM peak (1 GPU); µs per decode step"
+PREFILL_METRIC = "prefill attention TFLOP/s (4 D FLOPs per visible query-key pair; 1 GPU)"
 DEFAULT_WORKLOAD = "bf16_h32_d128_n128k"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
@@ -43,11 +45,22 @@ KERNEL_SOURCES = {
     "td_partial_kernel": ["td_partial.cu", "td_device.cuh", "td_internal.cuh"],
     "td_gqa_keys_kernel": ["td_gqa_keys.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
     "td_gqa_kernel": ["td_gqa.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
+    "td_prefill_kernel": ["td_prefill.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
 }
 
 
 def log(*a):
     print(*a, file=sys.stderr, flush=True)
+
+
+def measured_tensor_peak():
+    """Dense bf16 TFLOP/s measured by cuBLAS on this machine (burst), or the fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 def measured_peak():
@@ -215,9 +228,37 @@ def oracle_rate_gqa(inp, w, budget_s, min_s=0.0, threads=0):
     return bytes_once * passes / dt / 1e9, min(threads, w.H), desc, dt
 
 
+def oracle_rate_prefill(inp, w, budget_s, min_s=0.0, threads=0):
+    """The fp64 oracle on the last query rows of head 0 (the most keys each),
+    as many as fit the budget; returns (TFLOP/s, threads, description, s)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    threads = threads or cores
+    S, D = w.N, w.D
+    # ~1 GFLOP/s of fp64 per core on the plain loops
+    n_rows = int(max(threads, min(S, budget_s * 1e9 * threads / (4.0 * D * S))))
+    rows = list(range(S - n_rows, S))
+    q, k, v = (inp[x][:1, :1].cpu().contiguous() for x in ("q", "k", "v"))
+    sl = None if inp["slopes"] is None else inp["slopes"][:1].cpu()
+    flops_once = sum(4.0 * D * ((r + 1) if w.causal else S) for r in rows)
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.prefill(q, k, v, causal=w.causal, slopes=sl, rows=rows, threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            break
+    desc = ("%d query rows (the last of head 0) of a %d-token %s prefill (%s, D=%d), %d pass(es), "
+            "%d thread(s)" % (n_rows, S, "causal" if w.causal else "full", DTYPE_NAME[w.dtype],
+                              D, passes, threads))
+    return flops_once * passes / dt / 1e12, threads, desc, dt
+
+
 def oracle_rate(inp, w, budget_s, min_s=0.0, threads=0):
     """Time the fp64 oracle on (b,h) rows of a host copy of the workload;
     returns (GB/s, threads used, description, seconds)."""
+    if w.prefill:
+        return oracle_rate_prefill(inp, w, budget_s, min_s, threads)
     if w.kv_heads and w.kv_heads != w.H:
         return oracle_rate_gqa(inp, w, budget_s, min_s, threads)
     import oracle
@@ -432,6 +473,103 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# ------------------------------------------------------------------ prefill
+
+def run_prefill(args):
+    """A step is one td_prefill call over the whole workload (one kernel)."""
+    import long_context_attention_td_b200 as td
+
+    world, rank, local = dist_setup(args.gpus)
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    w = WORKLOADS[args.workload]
+    w = w.with_(seed=w.seed + 1000 * rank)
+    if args.n_keys:
+        w = w.with_(N=args.n_keys)
+    inp = make_inputs(w, dev)
+    q, k, v, slopes = inp["q"], inp["k"], inp["v"], inp["slopes"]
+    stream = torch.cuda.current_stream(dev)
+    out = torch.empty((w.B, w.H, w.N, w.D), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    flops = prefill_flops(w)
+
+    def step():
+        td.prefill(q, k, v, causal=w.causal, slopes=slopes, out=out, lse=lse, stream=stream)
+
+    sampler = ClockSampler(dev.index).start()
+    t_load0 = time.perf_counter()
+    for _ in range(args.warmup):
+        step()
+    td.check_device_error(stream=stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    launches0 = td.launch_count()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    launches = td.launch_count() - launches0
+    torch.cuda.synchronize(dev)
+    barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    while time.perf_counter() - t_load0 < 1.2:
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    td.check_device_error(stream=stream)
+    n_kt = min(args.steps, 20)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_kt)]
+    with torch.cuda.stream(stream):
+        for a, b in evs:
+            td.set_kernel_events(a, b)
+            step()
+        td.set_kernel_events(None, None)
+    torch.cuda.synchronize(dev)
+    kernel_name = td.last_kernel()
+    kernel_ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / n_kt, dev)
+    ms_max = reduce_max(ms_total, dev)
+    ms_per_step = ms_max / args.steps
+    flops_all = reduce_sum(flops * args.steps, dev)
+    peak, peak_kind = measured_tensor_peak()
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, used, desc, dt = oracle_rate_prefill(inp, w, budget_s=2.0, min_s=args.cpu_seconds)
+        cpu = {"value": round(rate, 6), "unit": "TFLOP/s", "cores": used, "kind": "oracle",
+               "sample": desc, "seconds": round(dt, 2), "host_cores": os.cpu_count()}
+    if rank == 0:
+        line = {
+            "metric": PREFILL_METRIC, "value": round(flops_all / (ms_max * 1e-3) / 1e12, 2),
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
+            "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
+            "config": {"workload": args.workload + ("" if not args.n_keys else "@S=%d" % w.N),
+                       "B": w.B, "H": w.H, "D": w.D, "S": w.N, "causal": w.causal,
+                       "alibi": w.alibi, "flops_per_step": flops,
+                       "l2": "no flush: q, k, v, out per step %.2f GB > 126 MB L2"
+                             % ((3 * 2 + 4) * w.B * w.H * w.N * w.D / 1e9),
+                       "parallelism": "replicas x%d" % world},
+            "gpu_launches": int(launches), "clocks": clocks,
+            "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
+                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                         "peak_kind": peak_kind, "traffic": profiled_traffic(args.workload,
+                                                                            kernel_name),
+                         "kernel": kernel_name, "algorithmic_flops_per_launch": flops},
+            "e2e": None, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 # ------------------------------------------- sequence-sharded (strong scaling)
 
 def run_sharded(args):
@@ -556,16 +694,17 @@ def run_reference(args):
         rates.append(r)
     dt = time.perf_counter() - t0
     value = sum(rates) / len(rates)
+    metric, unit = (PREFILL_METRIC, "TFLOP/s") if w.prefill else (METRIC, "GB/s")
     line = {
-        "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": world,
+        "metric": metric, "value": round(value, 6), "unit": unit, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * dt / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic", "impl": "reference",
         "config": {"workload": args.workload, "B": w.B, "H": w.H, "D": w.D, "N": w.N},
-        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": used,
+        "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": used,
                          "kind": "oracle", "sample": "per step: " + desc},
-        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+        "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -595,6 +734,8 @@ def main(argv=None):
         run_reference(args)
     elif args.shard_seq:
         run_sharded(args)
+    elif WORKLOADS[args.workload].prefill:
+        run_prefill(args)
     else:
         run_ours(args)
 

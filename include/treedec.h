@@ -223,6 +223,26 @@ TD_API td_status td_merge_shards(const float *states, int W, int B, int H, int D
                                  float *lse, td_stream stream);
 
 /*
+ * td_prefill -- attention of every query row of B*H sequences of S tokens
+ * (the step before decoding): for query i of head h,
+ *   s_ij = q_i . k_j D^-1/2 + slope_h (j - S + 1)  over keys j <= i (causal != 0)
+ *   or all keys (causal == 0); out_i = softmax_j(s_ij) . v, lse_i = ln sum_j e^s_ij.
+ * The bias is the ALiBi broadcast row of "ALiBi with causal=True unexpected
+ * bias?" over the whole sequence; the computation is the blockwise forward of
+ * "Flash Aandacht" (running max and sum per query row over key blocks, the
+ * running output rescaled by its old sum), on the tensor cores.
+ *   q, k, v  device [B,H,S,D] bf16 or fp16 (dtype), row-major, 16-byte aligned;
+ *   out      device fp32 [B,H,S,D], 16-byte aligned; lse device fp32 [B,H,S] or NULL;
+ *   alibi_slopes device fp32 [H] or NULL.
+ *   D in {64, 128}; S >= 1; B*H*ceil(S/128) < 2^31.
+ * Errors: TD_ERR_INVALID_ARG / TD_ERR_UNSUPPORTED before any launch; a bounded
+ * wait that ran out sets TD_DEVERR_WAIT_TIMEOUT (td_check_device_error).
+ */
+TD_API td_status td_prefill(const void *q, const void *k, const void *v, float *out, float *lse,
+                            int B, int H, int64_t S, int D, int causal,
+                            const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
+/*
  * td_auto_split -- the split heuristic: the number of parts (CTAs) for T =
  * B*H*N attended keys on a GPU with num_sms SMs: enough to fill every SM with
  * as many CTAs as fit at once, but no part smaller than 64 KiB of K+V and
@@ -334,7 +354,8 @@ TD_API void td_release_workspace(void);
  *
  * td_last_kernel -- name of the main kernel this thread's last successful
  * launch used ("td_partial_kernel", "td_gqa_keys_kernel", "td_gqa_kernel",
- * "td_tree_combine_kernel", "td_merge_shards_kernel", "td_empty_state_kernel";
+ * "td_tree_combine_kernel", "td_merge_shards_kernel", "td_empty_state_kernel",
+ * "td_prefill_kernel";
  * "" before the first).  Static storage.
  */
 TD_API uint64_t td_launch_count(void);

@@ -98,6 +98,8 @@ def lib():
     L.td_decode_shard.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, i64, i64, i32, vp, i32, vp]
     L.td_merge_shards.restype = i32
     L.td_merge_shards.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+    L.td_prefill.restype = i32
+    L.td_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, vp, i32, vp]
     L.td_launch_count.restype = ctypes.c_uint64
     L.td_launch_count.argtypes = []
     L.td_set_kernel_events.restype = i32
@@ -333,6 +335,28 @@ def check_device_error(workspace=None, stream=None):
     st = lib().td_check_device_error(ws, nbytes, ctypes.byref(bits), _stream(stream))
     if st != 0:
         raise TreeDecError(st, "kernel", "error bits 0x%x" % bits.value)
+
+
+def prefill(q, k, v, *, causal=True, slopes=None, out=None, lse=None, stream=None):
+    """Prefill attention of every query row: q, k, v [B,H,S,D] (bf16/fp16);
+    returns out fp32 [B,H,S,D] and lse fp32 [B,H,S]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev_tensor(t, n)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must all be [B,H,S,D]")
+    B, H, S, D = q.shape
+    if out is None:
+        out = torch.empty((B, H, S, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, S), dtype=torch.float32, device=q.device)
+    _dev_tensor(out, "out", torch.float32)
+    _dev_tensor(lse, "lse", torch.float32)
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    st = lib().td_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, S, D,
+                          1 if causal else 0, _ptr(slopes), DTYPE_CODE[q.dtype], _stream(stream))
+    _check(st, "td_prefill")
+    return out, lse
 
 
 def state_floats(B, H, D):

@@ -487,9 +487,84 @@ td_status gqa_impl(const GqaReq& r) {
     return cuda_status(launch_aux([&] { return td::launch_gqa_combine(r.D, p, r.stream); }));
 }
 
+// ------------------------------------------------------------------ prefill
+
+// 3-D map over [BH, S, D] elements, box {64 columns, 128 rows, 1}, 128-byte
+// swizzle; rows past S read as zero.
+td_status make_seq_map(CUtensorMap* map, const void* base, long long BH, long long S, int D,
+                       int dtype) {
+    PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return TD_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(S),
+                          static_cast<cuuint64_t>(BH)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(S) * D * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult rc = enc(map,
+                            dtype == TD_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                             : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                            3, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return rc == CUDA_SUCCESS ? TD_OK : TD_ERR_INVALID_ARG;
+}
+
+td_status prefill_validate(const void* q, const void* k, const void* v, const float* out,
+                           const float* lse, int B, int H, int64_t S, int D,
+                           const float* slopes, int dtype) {
+    if (!q || !k || !v || !out) return TD_ERR_INVALID_ARG;
+    if (dtype != TD_BF16 && dtype != TD_F16) return TD_ERR_UNSUPPORTED;
+    if (D != 64 && D != 128) return TD_ERR_UNSUPPORTED;
+    if (B < 1 || H < 1 || S < 1) return TD_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)) || (slopes && !aligned(slopes, 4)))
+        return TD_ERR_INVALID_ARG;
+    const long long BH = static_cast<long long>(B) * H;
+    // tensor-map coordinates are 32-bit; the grid is B*H*ceil(S/128) CTAs
+    if (S > 0x7fffffffLL || BH > 0x7fffffffLL || !mul_fits(BH, S) ||
+        BH * ((S + 127) / 128) > 0x7fffffffLL || !mul_fits(BH * S, static_cast<long long>(D) * 4))
+        return TD_ERR_INVALID_ARG;
+    return TD_OK;
+}
+
 }  // namespace
 
 extern "C" {
+
+td_status td_prefill(const void* q, const void* k, const void* v, float* out, float* lse, int B,
+                     int H, int64_t S, int D, int causal, const float* alibi_slopes,
+                     td_dtype dtype, td_stream stream) {
+    td_status st = prefill_validate(q, k, v, out, lse, B, H, S, D, alibi_slopes,
+                                    static_cast<int>(dtype));
+    if (st != TD_OK) return st;
+    int dev = 0, sms = 0;
+    st = current_device(&dev, &sms);
+    if (st != TD_OK) return st;
+    const long long BH = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv;
+    st = make_seq_map(&mq, q, BH, S, D, dtype);
+    if (st == TD_OK) st = make_seq_map(&mk, k, BH, S, D, dtype);
+    if (st == TD_OK) st = make_seq_map(&mv, v, BH, S, D, dtype);
+    if (st != TD_OK) return st;
+    const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    char* base = nullptr;
+    st = prepare_ws(dev, nullptr, 0, 0, td::kErrRegion, s, &base);
+    if (st != TD_OK) return st;
+    td::PrefillParams p;
+    p.out = out;
+    p.lse = lse;
+    p.slopes = alibi_slopes;
+    p.B = B;
+    p.H = H;
+    p.S = S;
+    p.causal = causal ? 1 : 0;
+    p.qscale2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(D)));
+    p.err = reinterpret_cast<int*>(base);
+    return cuda_status(launch_main(s, "td_prefill_kernel", [&] {
+        return td::launch_prefill(dev, static_cast<int>(dtype), D, p, mq, mk, mv, s);
+    }));
+}
+
 
 td_status td_decode_gqa(const void* q, const void* k, const void* v, float* out, float* lse, int B,
                         int Hq, int Hkv, int64_t N, int D, const int32_t* seqlens,

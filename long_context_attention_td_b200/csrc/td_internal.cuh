@@ -100,6 +100,22 @@ size_t partial_smem_bytes(int dtype, int D);
 // CTAs of the split-KV kernel that fit on one SM (static estimate from shared
 // memory and threads; matches the kernel's launch bounds).
 int partial_ctas_per_sm(int dtype, int D);
+// Prefill kernel (td_prefill.cu): every query row of B*H sequences of S tokens.
+struct PrefillParams {
+    float* out;              // [B, H, S, D]
+    float* lse;              // [B, H, S] or null
+    const float* slopes;     // [H] or null
+    int B, H;
+    int64_t S;
+    int causal;
+    float qscale2;           // D^-1/2 * log2(e)
+    int* err;
+};
+// Q, K, V tensor maps: 3-D [B*H, S, D], box {64, 128, 1}, 128-byte swizzle.
+cudaError_t launch_prefill(int device, int dtype, int D, const PrefillParams& p,
+                           const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                           cudaStream_t s);
+
 // Empty partial state (out 0, lse -inf) of `rows` (b,h) rows: a shard with no keys.
 cudaError_t launch_empty_state(float* out, float* lse, long long rows, int D, cudaStream_t s);
 // Merge W gathered shard states [W][rows*D | rows] into out[rows][D], lse[rows].

@@ -44,6 +44,8 @@ class Workload:
     spikes: int = 0
     seed: int = 1234
     kv_heads: int = 0           # grouped-query: key/value heads (0 = H, plain multi-head)
+    prefill: bool = False       # every query row of an N-token sequence (q, k, v [B,H,N,D])
+    causal: bool = True         # prefill: keys j <= i only
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -75,6 +77,13 @@ WORKLOADS = {
     # multi-query decode: 32 query heads over one kv head, 1M keys
     "mqa_bf16_h32_kv1_d128_n1m": Workload("mqa_bf16_h32_kv1_d128_n1m", torch.bfloat16, 1, 32,
                                           128, 1 << 20, seed=1240, kv_heads=1),
+    # causal prefill of an 8K-token prompt, 32 heads (tensor cores)
+    "prefill_bf16_h32_d128_s8k": Workload("prefill_bf16_h32_d128_s8k", torch.bfloat16, 1, 32,
+                                          128, 8192, seed=1241, prefill=True),
+    # batched causal prefill with the ALiBi row
+    "prefill_bf16_alibi_b4_h16_d128_s4k": Workload("prefill_bf16_alibi_b4_h16_d128_s4k",
+                                                   torch.bfloat16, 4, 16, 128, 4096, alibi=True,
+                                                   seed=1242, prefill=True),
 }
 
 
@@ -125,8 +134,28 @@ def make_gqa_inputs(w: Workload, Hkv: int, device="cpu"):
     return dict(q=q, k=k, v=v, slopes=slopes, seqlens=seqlens, seqlens_host=sl_host)
 
 
+def make_prefill_inputs(w: Workload, device="cpu"):
+    """Prefill inputs: q, k, v [B, H, N, D] drawn like make_inputs (q first)."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    B, H, D, N = w.B, w.H, w.D, w.N
+    q = _randn_rows(g, B * H * N, D, device, w.scale, w.dtype).view(B, H, N, D)
+    k = _randn_rows(g, B * H * N, D, device, w.scale, w.dtype).view(B, H, N, D)
+    v = _randn_rows(g, B * H * N, D, device, w.scale, w.dtype).view(B, H, N, D)
+    slopes = alibi_slopes(H, device) if w.alibi else None
+    return dict(q=q, k=k, v=v, slopes=slopes, seqlens=None, seqlens_host=None)
+
+
+def prefill_flops(w: Workload) -> float:
+    """Algorithmic FLOPs of a prefill: 4 D per visible (query, key) pair."""
+    pairs = w.N * (w.N + 1) / 2 if w.causal else float(w.N) * w.N
+    return 4.0 * w.D * pairs * w.B * w.H
+
+
 def make_inputs(w: Workload, device="cpu"):
     """Materialise a workload: dict(q, k, v, slopes, seqlens, seqlens_host)."""
+    if w.prefill:
+        return make_prefill_inputs(w, device)
     if w.kv_heads and w.kv_heads != w.H:
         return make_gqa_inputs(w, w.kv_heads, device)
     device = torch.device(device)

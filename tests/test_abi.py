@@ -169,3 +169,13 @@ def test_shard_entry_points_reject_bad_arguments(L):
     assert L.td_merge_shards(p, 0, 1, 1, 128, p, p, None) == INVALID
     assert L.td_merge_shards(p, 2, 1, 1, 1024, p, p, None) == INVALID
     assert L.td_merge_shards(None, 2, 1, 1, 128, p, p, None) == INVALID
+
+
+def test_prefill_rejects_bad_arguments(L):
+    p = ctypes.c_void_p(256)
+    odd = ctypes.c_void_p(258)
+    assert L.td_prefill(p, p, p, p, p, 1, 1, 128, 128, 1, None, 0, None) == UNSUPPORTED  # fp32
+    assert L.td_prefill(p, p, p, p, p, 1, 1, 128, 96, 1, None, 1, None) == UNSUPPORTED   # D
+    assert L.td_prefill(p, p, p, p, p, 1, 1, 0, 128, 1, None, 1, None) == INVALID        # S
+    assert L.td_prefill(odd, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID     # align
+    assert L.td_prefill(None, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID
