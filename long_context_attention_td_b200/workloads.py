@@ -45,6 +45,7 @@ class Workload:
     seed: int = 1234
     kv_heads: int = 0           # grouped-query: key/value heads (0 = H, plain multi-head)
     prefill: bool = False       # every query row of an N-token sequence (q, k, v [B,H,N,D])
+    kv_fp8: bool = False        # K/V as FP8 E4M3 codes (uint8) with per-head fp32 scales
     causal: bool = True         # prefill: keys j <= i only
 
     def with_(self, **kw) -> "Workload":
@@ -52,6 +53,9 @@ class Workload:
 
     @property
     def elt(self) -> int:
+        """Bytes per K/V element."""
+        if self.kv_fp8:
+            return 1
         return torch.tensor([], dtype=self.dtype).element_size()
 
 
@@ -77,6 +81,9 @@ WORKLOADS = {
     # multi-query decode: 32 query heads over one kv head, 1M keys
     "mqa_bf16_h32_kv1_d128_n1m": Workload("mqa_bf16_h32_kv1_d128_n1m", torch.bfloat16, 1, 32,
                                           128, 1 << 20, seed=1240, kv_heads=1),
+    # the bench decode shape with an FP8 (E4M3) K/V cache and per-head scales
+    "fp8kv_h32_d128_n128k": Workload("fp8kv_h32_d128_n128k", torch.bfloat16, 1, 32, 128, 131072,
+                                     seed=1243, kv_fp8=True),
     # causal prefill of an 8K-token prompt, 32 heads (tensor cores)
     "prefill_bf16_h32_d128_s8k": Workload("prefill_bf16_h32_d128_s8k", torch.bfloat16, 1, 32,
                                           128, 8192, seed=1241, prefill=True),
@@ -152,8 +159,47 @@ def prefill_flops(w: Workload) -> float:
     return 4.0 * w.D * pairs * w.B * w.H
 
 
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3(x: torch.Tensor):
+    """Per-head FP8 E4M3 codes of x [B,H,N,D] (fp32): scale_h = amax_h / 448,
+    codes = round-to-nearest(x / scale_h), returned as their uint8 bits with the
+    fp32 scales [H].  This prepares a cache the way a serving stack stores it;
+    the attention arithmetic on it is the library's (and the oracle's)."""
+    amax = x.abs().amax(dim=(0, 2, 3)).clamp_min(1e-30)
+    scale = (amax / E4M3_MAX).to(torch.float32)
+    y = (x / scale[None, :, None, None]).clamp(-E4M3_MAX, E4M3_MAX)
+    return y.to(torch.float8_e4m3fn).view(torch.uint8), scale
+
+
+def make_fp8_inputs(w: Workload, device="cpu"):
+    """q [B,H,1,D] in w.dtype; k, v [B,H,N,D] FP8 E4M3 codes (uint8) drawn as
+    N(0,1)*scale in fp32 then quantised per head; k_scale, v_scale [H]."""
+    device = torch.device(device)
+    g = torch.Generator(device=device).manual_seed(w.seed)
+    B, H, D, N = w.B, w.H, w.D, w.N
+    qf = torch.randn((B, H, 1, D), generator=g, device=device, dtype=torch.float32)
+    if w.scale != 1.0:
+        qf.mul_(w.scale)
+    q = qf.to(w.dtype)
+    kf = _randn_rows(g, B * H * N, D, device, w.scale, torch.float32).view(B, H, N, D)
+    k, k_scale = quantize_e4m3(kf)
+    del kf
+    vf = _randn_rows(g, B * H * N, D, device, w.scale, torch.float32).view(B, H, N, D)
+    v, v_scale = quantize_e4m3(vf)
+    del vf
+    sl_host = seqlens_for(w)
+    slopes = alibi_slopes(H, device) if w.alibi else None
+    seqlens = sl_host.to(device) if sl_host is not None else None
+    return dict(q=q, k=k, v=v, k_scale=k_scale, v_scale=v_scale, slopes=slopes,
+                seqlens=seqlens, seqlens_host=sl_host)
+
+
 def make_inputs(w: Workload, device="cpu"):
     """Materialise a workload: dict(q, k, v, slopes, seqlens, seqlens_host)."""
+    if w.kv_fp8:
+        return make_fp8_inputs(w, device)
     if w.prefill:
         return make_prefill_inputs(w, device)
     if w.kv_heads and w.kv_heads != w.H:

@@ -21,7 +21,7 @@ import numpy as np
 
 from . import build as _build
 
-_F32, _BF16, _F16 = 0, 1, 2
+_F32, _BF16, _F16, _F64 = 0, 1, 2, 3
 _lib = None
 
 
@@ -37,6 +37,8 @@ def lib():
         L.or_decode_bf16.argtypes = [ctypes.c_uint16]
         L.or_decode_f16.restype = ctypes.c_double
         L.or_decode_f16.argtypes = [ctypes.c_uint16]
+        L.or_decode_e4m3.restype = ctypes.c_double
+        L.or_decode_e4m3.argtypes = [ctypes.c_uint8]
         L.or_alibi_bias.restype = ctypes.c_double
         L.or_alibi_bias.argtypes = [ctypes.c_double, ctypes.c_int64, ctypes.c_int64]
         L.or_attend_one.restype = ctypes.c_int
@@ -77,14 +79,16 @@ def _code_and_buf(x):
             if t.device.type != "cpu":
                 raise ValueError("oracle inputs must be CPU tensors")
             t = t.contiguous()
-            code = {torch.float32: _F32, torch.bfloat16: _BF16, torch.float16: _F16}.get(t.dtype)
+            code = {torch.float32: _F32, torch.bfloat16: _BF16, torch.float16: _F16,
+                    torch.float64: _F64}.get(t.dtype)
             if code is None:
                 raise TypeError("unsupported dtype %s" % t.dtype)
             return code, t, t.data_ptr()
     except ImportError:
         pass
     a = np.ascontiguousarray(x)
-    code = {np.dtype(np.float32): _F32, np.dtype(np.float16): _F16}.get(a.dtype)
+    code = {np.dtype(np.float32): _F32, np.dtype(np.float16): _F16,
+            np.dtype(np.float64): _F64}.get(a.dtype)
     if code is None:
         raise TypeError("unsupported dtype %s" % a.dtype)
     return code, a, a.ctypes.data
@@ -253,6 +257,21 @@ def decode_bf16(bits):
 
 def decode_f16(bits):
     return lib().or_decode_f16(int(bits))
+
+
+def decode_e4m3(bits):
+    return lib().or_decode_e4m3(int(bits))
+
+
+def dequant_e4m3(x8, scales):
+    """FP8 E4M3 cache [B,H,N,D] (uint8 bits) times per-head scales [H] as fp64
+    (exact: a 4-bit by 24-bit significand product)."""
+    lut = np.array([decode_e4m3(b) for b in range(256)], dtype=np.float64)
+    a = np.asarray(x8.cpu() if hasattr(x8, "cpu") else x8)
+    if a.dtype != np.uint8:
+        raise TypeError("FP8 caches are passed as their uint8 bits")
+    sc = np.asarray(scales.cpu() if hasattr(scales, "cpu") else scales, dtype=np.float32)
+    return lut[a] * sc.astype(np.float64)[None, :, None, None]
 
 
 def alibi_bias(slope, j, n):

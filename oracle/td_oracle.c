@@ -47,6 +47,7 @@
 #define OR_F32 0
 #define OR_BF16 1
 #define OR_F16 2
+#define OR_F64 3 /* already-widened values (e.g. dequantised FP8 caches) */
 
 /* ---------------------------------------------------------------- decoders */
 
@@ -73,7 +74,27 @@ double or_decode_f16(uint16_t h) {
     return sign ? -v : v;
 }
 
+/*
+ * FP8 E4M3 (the "fn" variant of the OCP 8-bit floating point formats): 1 sign
+ * bit, 4 exponent bits (bias 7), 3 fraction bits; exponent 0 is subnormal
+ * (m/8 * 2^-6); no infinities; S.1111.111 is NaN; the largest value is 448.
+ */
+double or_decode_e4m3(uint8_t b) {
+    int sign = (b >> 7) & 1;
+    int e = (b >> 3) & 0xf;
+    int m = b & 7;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -9); /* m/8 * 2^-6 */
+    else if (e == 15 && m == 7)
+        v = NAN;
+    else
+        v = ldexp((double)(m + 8), e - 10); /* (1 + m/8) * 2^(e-7) */
+    return sign ? -v : v;
+}
+
 static double load_elem(const void *base, int64_t idx, int dtype) {
+    if (dtype == OR_F64) return ((const double *)base)[idx];
     if (dtype == OR_F32) return (double)((const float *)base)[idx];
     uint16_t h = ((const uint16_t *)base)[idx];
     return dtype == OR_BF16 ? or_decode_bf16(h) : or_decode_f16(h);
@@ -333,7 +354,7 @@ static void *worker(void *arg) {
 
 static int run(job_t *J, int threads) {
     if (!J->q || !J->k || !J->v || !J->out || !J->lse) return -1;
-    if (J->dtype < OR_F32 || J->dtype > OR_F16 || J->B <= 0 || J->H <= 0 || J->D <= 0 ||
+    if (J->dtype < OR_F32 || J->dtype > OR_F64 || J->B <= 0 || J->H <= 0 || J->D <= 0 ||
         J->Nmax < 0 || J->n_bh < 0 || J->Hkv <= 0 || J->H % J->Hkv != 0)
         return -1;
     if (J->seqlens)
@@ -468,7 +489,7 @@ static void *prefill_worker(void *arg) {
 int or_prefill(const void *q, const void *k, const void *v, int dtype, int B, int H, int64_t S,
                int D, int causal, const float *slopes, const int64_t *rows, int64_t n_rows,
                double *out, double *lse, int threads) {
-    if (!q || !k || !v || !out || !lse || dtype < OR_F32 || dtype > OR_F16 || B <= 0 ||
+    if (!q || !k || !v || !out || !lse || dtype < OR_F32 || dtype > OR_F64 || B <= 0 ||
         H <= 0 || S <= 0 || D <= 0 || n_rows < 0)
         return -1;
     prefill_job_t J = {q, k, v, dtype, B, H, D, causal ? 1 : 0, S, slopes, rows,

@@ -549,3 +549,58 @@ def test_prefill_first_row_closed_form_and_row_selection():
                               rows=rows)
     np.testing.assert_array_equal(os_, o[rows])
     np.testing.assert_array_equal(ls_, l[rows])
+
+
+# --------------------------------------------------------- FP8 (E4M3) caches
+
+def test_e4m3_decoder_matches_torch_on_every_code():
+    """Library pin: torch's float8_e4m3fn widening, all 256 codes."""
+    bits = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = bits.view(torch.float8_e4m3fn).double().numpy()
+    got = np.array([oracle.decode_e4m3(b) for b in range(256)])
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+    ok = ~np.isnan(ref)
+    np.testing.assert_array_equal(got[ok], ref[ok])
+
+
+def test_e4m3_decoder_closed_forms():
+    assert oracle.decode_e4m3(0x7E) == 448.0           # largest finite
+    assert oracle.decode_e4m3(0x01) == 2.0 ** -9        # smallest subnormal
+    assert oracle.decode_e4m3(0x08) == 2.0 ** -6        # smallest normal
+    assert oracle.decode_e4m3(0x38) == 1.0
+    assert oracle.decode_e4m3(0xB8) == -1.0
+    assert math.isnan(oracle.decode_e4m3(0x7F)) and math.isnan(oracle.decode_e4m3(0xFF))
+    assert oracle.decode_e4m3(0x00) == 0.0 and math.copysign(1, oracle.decode_e4m3(0x80)) < 0
+
+
+def test_fp64_inputs_agree_with_fp32_inputs():
+    """The widened-input path reads the same numbers as the fp32 path."""
+    B, H, N, D = 1, 3, 41, 16
+    q = _rand((B, H, 1, D), torch.float32, 221)
+    k = _rand((B, H, N, D), torch.float32, 222)
+    v = _rand((B, H, N, D), torch.float32, 223)
+    slopes = np.array([0.1, 0.2, 0.3], dtype=np.float32)
+    a = oracle.full(q, k, v, slopes=slopes)
+    b = oracle.full(q.double(), k.double(), v.double(), slopes=slopes)
+    np.testing.assert_array_equal(a[0], b[0])
+    np.testing.assert_array_equal(a[1], b[1])
+
+
+def test_fp8_cache_attention_is_attention_on_the_dequantised_cache():
+    """An FP8 cache with per-head scales means K = e4m3(k8) * k_scale[h] (and V
+    alike); fp64 SDPA on those dequantised values is the library pin."""
+    B, H, N, D = 2, 2, 50, 32
+    g = torch.Generator().manual_seed(231)
+    q = torch.randn((B, H, 1, D), generator=g).to(torch.bfloat16)
+    k8 = torch.randint(0, 256, (B, H, N, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    v8 = torch.randint(0, 256, (B, H, N, D), generator=g, dtype=torch.int32).to(torch.uint8)
+    k8[(k8 & 0x7F) == 0x7F] = 0x38   # no NaN codes in a cache
+    v8[(v8 & 0x7F) == 0x7F] = 0x38
+    ks = np.array([0.01, 0.002], dtype=np.float32)
+    vs = np.array([0.5, 0.03125], dtype=np.float32)
+    K = oracle.dequant_e4m3(k8, ks)
+    V = oracle.dequant_e4m3(v8, vs)
+    o, l = oracle.full(q.double(), torch.from_numpy(K), torch.from_numpy(V))
+    ref = torch.nn.functional.scaled_dot_product_attention(q.double(), torch.from_numpy(K),
+                                                           torch.from_numpy(V))
+    np.testing.assert_allclose(o, ref.reshape(B * H, D).numpy(), rtol=0, atol=1e-12)
