@@ -254,11 +254,38 @@ def oracle_rate_prefill(inp, w, budget_s, min_s=0.0, threads=0):
     return flops_once * passes / dt / 1e12, threads, desc, dt
 
 
+def oracle_rate_fp8(inp, w, budget_s, min_s=0.0, threads=0):
+    """The fp64 oracle on the first keys of every head of batch 0 of an FP8
+    cache, dequantised (outside the timed region) to the fp64 values it
+    stands for; GB/s counts the FP8 bytes those keys occupy."""
+    import oracle
+    cores = os.cpu_count() or 1
+    threads = threads or cores
+    H, D = w.H, w.D
+    nk = max(1024, min(w.N, int(budget_s * 0.25e9 * min(threads, H) / (2 * D * H))))
+    q = inp["q"][:1].double().cpu()
+    K = torch.from_numpy(oracle.dequant_e4m3(inp["k"][:1, :, :nk].cpu(), inp["k_scale"]))
+    V = torch.from_numpy(oracle.dequant_e4m3(inp["v"][:1, :, :nk].cpu(), inp["v_scale"]))
+    bytes_once = 2 * H * nk * D  # one byte per FP8 element
+    passes, t0 = 0, time.perf_counter()
+    while True:
+        oracle.full(q, K, V, threads=threads)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= min_s:
+            break
+    desc = ("%d heads x %d keys of an FP8 cache (D=%d, dequantised to fp64 before timing), "
+            "%d pass(es), %d thread(s)" % (H, nk, D, passes, min(threads, H)))
+    return bytes_once * passes / dt / 1e9, min(threads, H), desc, dt
+
+
 def oracle_rate(inp, w, budget_s, min_s=0.0, threads=0):
     """Time the fp64 oracle on (b,h) rows of a host copy of the workload;
     returns (GB/s, threads used, description, seconds)."""
     if w.prefill:
         return oracle_rate_prefill(inp, w, budget_s, min_s, threads)
+    if w.kv_fp8:
+        return oracle_rate_fp8(inp, w, budget_s, min_s, threads)
     if w.kv_heads and w.kv_heads != w.H:
         return oracle_rate_gqa(inp, w, budget_s, min_s, threads)
     import oracle
@@ -334,7 +361,11 @@ def run_ours(args):
                               total_keys if inp["seqlens"] is not None else -1)
 
     def step():
-        if gqa:
+        if w.kv_fp8:
+            td.decode_fp8(q, k, v, inp["k_scale"], inp["v_scale"], seqlens=inp["seqlens"],
+                          seqlens_host=inp["seqlens_host"], slopes=inp["slopes"],
+                          n_split=n_split, out=out, lse=lse, stream=stream)
+        elif gqa:
             td.decode_gqa(q, k, v, seqlens=inp["seqlens"], seqlens_host=inp["seqlens_host"],
                           slopes=inp["slopes"], n_split=n_split, out=out, lse=lse, stream=stream)
         elif inp["seqlens"] is not None:
@@ -398,7 +429,7 @@ def run_ours(args):
 
     # end to end through the host-buffer entry point (pinned host inputs)
     e2e = None
-    if not args.no_e2e and not gqa:
+    if not args.no_e2e and not gqa and not w.kv_fp8:
         qh = q.cpu().pin_memory()
         kh = k.cpu().pin_memory()
         vh = v.cpu().pin_memory()
@@ -456,7 +487,9 @@ def run_ours(args):
             "pct_of_nominal_8tbs": round(100 * per_gpu / NOMINAL_HBM_GBS, 2),
             "tokens_of_kv_per_s": round(total_keys * world / (ms_per_step * 1e-3), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
+            "dtype": "f32", "input_dtype": (DTYPE_NAME[w.dtype] + " q, e4m3 k/v (f16 products)"
+                                            if w.kv_fp8 else DTYPE_NAME[w.dtype]),
+            "data": "synthetic",
             "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
                        "B": B, "H": H, "kv_heads": w.kv_heads or H, "D": D, "N": N,
                        "ragged": w.ragged is not None, "alibi": w.alibi,

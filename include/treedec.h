@@ -91,6 +91,24 @@ TD_API td_status td_decode(const void *q, const void *k, const void *v, float *o
                     const float *alibi_slopes, td_dtype dtype, td_stream stream);
 
 /*
+ * td_decode_fp8 -- td_decode / td_decode_varlen over an FP8 K/V cache: k8, v8
+ * device [B,H,Nmax,D] bytes holding OCP FP8 E4M3 codes (1 sign, 4 exponent
+ * bits with bias 7, 3 fraction bits; no infinities), dequantised per head as
+ * K = e4m3(k8) * k_scale[h], V = e4m3(v8) * v_scale[h] (k_scale, v_scale
+ * device fp32 [H]).  The result is the attention of q (q_dtype TD_BF16 or
+ * TD_F16) over those dequantised K, V.  seqlens/seqlens_host as
+ * td_decode_varlen (NULL: every sequence has Nmax keys); other arguments and
+ * errors as td_decode.  Arithmetic: q.k and p v are multiply-added in half
+ * precision (8-term chains for q.k with q pre-scaled by a power of two; at most
+ * a tile's rows for p v, then fp32), softmax and sums in fp32.
+ */
+TD_API td_status td_decode_fp8(const void *q, const void *k8, const void *v8, const float *k_scale,
+                               const float *v_scale, float *out, float *lse, int B, int H,
+                               int64_t Nmax, int D, const int32_t *seqlens,
+                               const int32_t *seqlens_host, int n_split,
+                               const float *alibi_slopes, td_dtype q_dtype, td_stream stream);
+
+/*
  * td_decode_varlen -- as td_decode for a batch of sequences of different
  * lengths stored padded: k, v [B,H,Nmax,D]; sequence b attends to its first
  * seqlens[b] keys and the ALiBi term uses n = seqlens[b].
@@ -355,7 +373,7 @@ TD_API void td_release_workspace(void);
  * td_last_kernel -- name of the main kernel this thread's last successful
  * launch used ("td_partial_kernel", "td_gqa_keys_kernel", "td_gqa_kernel",
  * "td_tree_combine_kernel", "td_merge_shards_kernel", "td_empty_state_kernel",
- * "td_prefill_kernel";
+ * "td_prefill_kernel", "td_partial_kernel (fp8 kv)";
  * "" before the first).  Static storage.
  */
 TD_API uint64_t td_launch_count(void);

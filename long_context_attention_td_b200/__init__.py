@@ -98,6 +98,9 @@ def lib():
     L.td_decode_shard.argtypes = [vp, vp, vp, vp, i32, i32, i64, i32, i64, i64, i32, vp, i32, vp]
     L.td_merge_shards.restype = i32
     L.td_merge_shards.argtypes = [vp, i32, i32, i32, i32, vp, vp, vp]
+    L.td_decode_fp8.restype = i32
+    L.td_decode_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i64, i32, vp, vp, i32, vp,
+                                i32, vp]
     L.td_prefill.restype = i32
     L.td_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, vp, i32, vp]
     L.td_launch_count.restype = ctypes.c_uint64
@@ -172,6 +175,39 @@ def decode(q, k, v, *, slopes=None, n_split=0, out=None, lse=None, stream=None):
     st = lib().td_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
                          int(n_split), _ptr(slopes), DTYPE_CODE[q.dtype], _stream(stream))
     _check(st, "td_decode")
+    return out, lse
+
+
+def decode_fp8(q, k8, v8, k_scale, v_scale, *, seqlens=None, seqlens_host=None, slopes=None,
+               n_split=0, out=None, lse=None, stream=None):
+    """Decode over an FP8 E4M3 K/V cache: k8, v8 [B,H,Nmax,D] uint8 codes (or
+    torch.float8_e4m3fn), dequantised per head by k_scale, v_scale fp32 [H];
+    q [B,H,1,D] bf16 or fp16.  Returns (out [B,H,1,D], lse [B,H,1]) fp32."""
+    k8 = k8.view(torch.uint8) if k8.dtype == torch.float8_e4m3fn else k8
+    v8 = v8.view(torch.uint8) if v8.dtype == torch.float8_e4m3fn else v8
+    _dev_tensor(q, "q")
+    _dev_tensor(k8, "k8", torch.uint8)
+    _dev_tensor(v8, "v8", torch.uint8)
+    _dev_tensor(k_scale, "k_scale", torch.float32)
+    _dev_tensor(v_scale, "v_scale", torch.float32)
+    if q.dim() != 4 or k8.dim() != 4 or v8.dim() != 4 or k8.shape != v8.shape:
+        raise ValueError("expected q [B,H,1,D], k8 and v8 [B,H,N,D]")
+    B, H, _, D = q.shape
+    N = int(k8.shape[2])
+    if tuple(k8.shape) != (B, H, N, D) or q.shape[2] != 1:
+        raise ValueError("expected q [B,H,1,D], k8 and v8 [B,H,N,D]")
+    if k_scale.numel() != H or v_scale.numel() != H:
+        raise ValueError("k_scale and v_scale hold one scale per head")
+    if seqlens is not None:
+        _dev_tensor(seqlens, "seqlens", torch.int32)
+    sh = None if seqlens_host is None else seqlens_host.to(torch.int32).contiguous().cpu()
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    out, lse = _outputs(q, B, H, D, out, lse)
+    st = lib().td_decode_fp8(_ptr(q), _ptr(k8), _ptr(v8), _ptr(k_scale), _ptr(v_scale),
+                             _ptr(out), _ptr(lse), B, H, N, D, _ptr(seqlens), _ptr(sh),
+                             int(n_split), _ptr(slopes), DTYPE_CODE[q.dtype], _stream(stream))
+    _check(st, "td_decode_fp8")
     return out, lse
 
 

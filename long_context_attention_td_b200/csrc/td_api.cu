@@ -105,7 +105,7 @@ td_status cuda_status(cudaError_t e) {
 }
 
 bool dtype_ok(int t) { return t == TD_F32 || t == TD_BF16 || t == TD_F16; }
-int elt_size(int t) { return t == TD_F32 ? 4 : 2; }
+int elt_size(int t) { return t == TD_F32 ? 4 : (t == td::kE4M3 ? 1 : 2); }
 bool d_ok(int D) { return D == 64 || D == 128 || D == 256 || D == 512; }
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -223,6 +223,11 @@ struct Req {
     size_t ws_bytes;
     cudaStream_t stream;
     long long alibi_off = 0;  // ALiBi position shift of a shard (see td_decode_shard)
+    // FP8 K/V cache: kv_dtype = td::kE4M3 with per-head scales; -1: K/V of type dtype
+    int kv_dtype = -1;
+    const float* k_scale = nullptr;
+    const float* v_scale = nullptr;
+    int kv() const { return kv_dtype < 0 ? dtype : kv_dtype; }
 };
 
 td_status validate(const Req& r) {
@@ -242,6 +247,14 @@ td_status validate(const Req& r) {
     if (r.seqlens_host)
         for (int b = 0; b < r.B; ++b)
             if (r.seqlens_host[b] < 0 || r.seqlens_host[b] > r.N) return TD_ERR_INVALID_ARG;
+    if (r.kv_dtype == td::kE4M3) {
+        // FP8 cache: q in half precision, both scales given
+        if (r.dtype != TD_BF16 && r.dtype != TD_F16) return TD_ERR_UNSUPPORTED;
+        if (!r.k_scale || !r.v_scale || !aligned(r.k_scale, 4) || !aligned(r.v_scale, 4))
+            return TD_ERR_INVALID_ARG;
+    } else if (r.kv_dtype >= 0 && r.kv_dtype != r.dtype) {
+        return TD_ERR_UNSUPPORTED;
+    }
     return TD_OK;
 }
 
@@ -258,7 +271,7 @@ long long plan_parts(const Req& r, int num_sms) {
     const long long bound = static_cast<long long>(r.B) * r.H * r.N;
     const long long known = known_keys(r);
     const long long T = known >= 0 ? known : bound;
-    long long P = r.parts > 0 ? r.parts : auto_parts(T, r.D, r.dtype, num_sms);
+    long long P = r.parts > 0 ? r.parts : auto_parts(T, r.D, r.kv(), num_sms);
     const long long cap = T > 0 ? T : 1;
     if (P > cap) P = cap;
     if (P > 0x7fffffffLL) P = 0x7fffffffLL;
@@ -296,6 +309,12 @@ td_status decode_impl(const Req& r) {
     p.tickets = reinterpret_cast<int*>(base + td::kErrRegion);
     p.part = reinterpret_cast<float*>(base + td::kErrRegion + ticket_region(BH));
     p.alibi_off = r.alibi_off;
+    p.k_scale = r.k_scale;
+    p.v_scale = r.v_scale;
+    if (r.kv() == td::kE4M3)
+        return cuda_status(launch_main(r.stream, "td_partial_kernel (fp8 kv)", [&] {
+            return td::launch_partial_fp8(dev, r.dtype, r.D, p, r.stream);
+        }));
     return cuda_status(launch_main(r.stream, "td_partial_kernel", [&] {
         return td::launch_partial(dev, r.dtype, r.D, p, r.stream);
     }));
@@ -649,6 +668,24 @@ td_status td_decode_ws(const void* q, const void* k, const void* v, float* out, 
     Req r{q, k, v, out, lse, B, H, N, D, seqlens, seqlens_host, parts, alibi_slopes,
           static_cast<int>(dtype), workspace, workspace_bytes,
           reinterpret_cast<cudaStream_t>(stream)};
+    return decode_impl(r);
+}
+
+td_status td_decode_fp8(const void* q, const void* k8, const void* v8, const float* k_scale,
+                        const float* v_scale, float* out, float* lse, int B, int H, int64_t Nmax,
+                        int D, const int32_t* seqlens, const int32_t* seqlens_host, int n_split,
+                        const float* alibi_slopes, td_dtype q_dtype, td_stream stream) {
+    if (n_split < 0) return TD_ERR_INVALID_ARG;
+    long long parts = 0;
+    if (n_split > 0) {
+        const long long per = (!seqlens && n_split > Nmax) ? Nmax : n_split;
+        parts = static_cast<long long>(B) * H * (per > 0 ? per : 1);
+    }
+    Req r{q, k8, v8, out, lse, B, H, Nmax, D, seqlens, seqlens_host, parts, alibi_slopes,
+          static_cast<int>(q_dtype), nullptr, 0, reinterpret_cast<cudaStream_t>(stream)};
+    r.kv_dtype = td::kE4M3;
+    r.k_scale = k_scale;
+    r.v_scale = v_scale;
     return decode_impl(r);
 }
 

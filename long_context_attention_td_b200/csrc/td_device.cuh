@@ -148,6 +148,25 @@ struct Elem<__nv_bfloat16> {
     }
 };
 
+// FP8 E4M3 storage element (K/V caches only): one byte; the kernels convert
+// pairs with cvt.rn.f16x2.e4m3x2 and multiply-add them in half precision.
+struct E4M3 {
+    unsigned char bits;
+};
+template <>
+struct Elem<E4M3> {
+    static constexpr int kVec = 16;  // elements per 16 B
+};
+
+// two E4M3 values (low byte -> low half) as an f16x2 word
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
+    uint32_t r;
+    asm("{\n\t.reg .b16 t;\n\tcvt.u16.u32 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}"
+        : "=r"(r)
+        : "r"(two));
+    return r;
+}
+
 template <>
 struct Elem<__half> {
     static constexpr int kVec = 8;

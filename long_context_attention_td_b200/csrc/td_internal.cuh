@@ -9,7 +9,7 @@
 namespace td {
 
 // Element types (same numbering as td_dtype).
-enum : int { kF32 = 0, kBF16 = 1, kF16 = 2 };
+enum : int { kF32 = 0, kBF16 = 1, kF16 = 2, kE4M3 = 3 };  // kE4M3: K/V storage only
 
 // Shape of the split-KV kernel's pipeline (compile-time; the defaults are the
 // tuned values, the macros exist for tuning sweeps).
@@ -61,6 +61,8 @@ struct PartialParams {
     int* err;                // error word
     int64_t alibi_off;       // ALiBi position of key j is j - n + 1 + alibi_off (0: the
                              // sequence is whole; a shard adds its place in the full one)
+    const float* k_scale;    // FP8 K/V: per-head dequantisation scales [H] (else null)
+    const float* v_scale;
 };
 
 // Grouped-query kernel (td_gqa.cu): Hq = G * Hkv query heads over Hkv kv heads.
@@ -95,7 +97,11 @@ size_t gqa_keys_smem_bytes(int G);
 cudaError_t launch_gqa_keys(int device, int dtype, const GqaParams& p, const CUtensorMap& mk,
                             const CUtensorMap& mv, cudaStream_t s);
 
-// Dynamic shared memory of the split-KV kernel for (dtype, D).
+// The split-KV kernel over an FP8 E4M3 K/V cache, q of type q_dtype (kBF16, kF16).
+cudaError_t launch_partial_fp8(int device, int q_dtype, int D, const PartialParams& p,
+                               cudaStream_t s);
+
+// Dynamic shared memory of the split-KV kernel for (K/V dtype, D).
 size_t partial_smem_bytes(int dtype, int D);
 // CTAs of the split-KV kernel that fit on one SM (static estimate from shared
 // memory and threads; matches the kernel's launch bounds).

@@ -24,6 +24,7 @@
 // holding 16 bytes of q, k, v and its slice of the fp32 accumulator; the dot
 // product is finished with xor shuffles inside the group.
 #include <atomic>
+#include <type_traits>
 
 #include "td_device.cuh"
 #include "td_internal.cuh"
@@ -145,9 +146,28 @@ struct SlotAcc {
 
 constexpr int kBarConsumers = 1;
 
-template <typename E, int D>
+// 16 E4M3 keys of a lane's slice (one 16-byte word) dotted with its q slice in
+// half precision: 8 chained f16x2 fused multiply-adds (q pre-scaled by a power
+// of two so every partial stays below 2^15).
+__device__ __forceinline__ float dot16_e4m3(const __half2 (&qh)[8], const uint4 w) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+    __half2 acc = __float2half2_rn(0.f);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t lo = e4m3x2_to_f16x2(ws[i] & 0xffffu);
+        const uint32_t hi = e4m3x2_to_f16x2(ws[i] >> 16);
+        acc = __hfma2(qh[2 * i], *reinterpret_cast<const __half2*>(&lo), acc);
+        acc = __hfma2(qh[2 * i + 1], *reinterpret_cast<const __half2*>(&hi), acc);
+    }
+    return __low2float(acc) + __high2float(acc);
+}
+
+// EQ: type of q; E: type of the K/V rows (EQ, or E4M3 for an FP8 cache).
+template <typename EQ, typename E, int D>
 __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel(const PartialParams p) {
     using C = Cfg<E, D>;
+    constexpr bool kFp8 = std::is_same<E, E4M3>::value;
+    static_assert(kFp8 || std::is_same<E, EQ>::value, "q and K/V share a type unless K/V is FP8");
     extern __shared__ __align__(1024) unsigned char smem[];
     __shared__ __align__(8) uint64_t full_bar[kStages];
     __shared__ __align__(8) uint64_t empty_bar[kStages];
@@ -305,14 +325,41 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         // to the finished dot product
         float qf[C::kNV][C::kVec];
         {
-            const E* qrow = static_cast<const E*>(p.q) + bh * D;
+            const EQ* qrow = static_cast<const EQ*>(p.q) + bh * D;
+            constexpr int kQV = Elem<EQ>::kVec;  // q elements per 16-byte load
 #pragma unroll
             for (int u = 0; u < C::kNV; ++u)
-                Elem<E>::to_f32(
-                    __ldg(reinterpret_cast<const uint4*>(qrow + (u * C::kG + lig) * C::kVec)),
-                    qf[u]);
+#pragma unroll
+                for (int part = 0; part < C::kVec / kQV; ++part)
+                    Elem<EQ>::to_f32(__ldg(reinterpret_cast<const uint4*>(
+                                         qrow + (u * C::kG + lig) * C::kVec + part * kQV)),
+                                     qf[u] + part * kQV);
         }
-        const float qscale2 = p.qscale2;
+        float qscale2 = p.qscale2;
+        // FP8 cache: q in half precision, scaled by 2^e so that |q| 2^e < 8 and
+        // each 8-term partial of q . k (|k| <= 448) stays below 2^15; the dot
+        // product is taken back by 2^-e, and the per-head key scale joins the
+        // score scale
+        __half2 qh[C::kNV][C::kVec / 2];
+        float qinv = 1.f;
+        if constexpr (kFp8) {
+            float amax = 0.f;
+#pragma unroll
+            for (int u = 0; u < C::kNV; ++u)
+#pragma unroll
+                for (int x = 0; x < C::kVec; ++x) amax = fmaxf(amax, fabsf(qf[u][x]));
+            int ex = 0;
+            frexpf(amax, &ex);                       // amax < 2^ex
+            const int e = amax > 0.f ? max(-24, min(24, 3 - ex)) : 0;
+            const float up = ldexpf(1.f, e);
+            qinv = ldexpf(1.f, -e);
+#pragma unroll
+            for (int u = 0; u < C::kNV; ++u)
+#pragma unroll
+                for (int x = 0; x < C::kVec / 2; ++x)
+                    qh[u][x] = __floats2half2_rn(qf[u][2 * x] * up, qf[u][2 * x + 1] * up);
+            qscale2 *= __ldg(p.k_scale + w.h);
+        }
         const bool has_bias = p.slopes != nullptr;
         const float slope2 = has_bias ? __ldg(p.slopes + w.h) * kLog2e : 0.f;
         const long long pos0 = 1 - w.len + p.alibi_off;   // ALiBi position of key 0
@@ -341,11 +388,17 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 if (row < rows) {
 #pragma unroll
                     for (int u = 0; u < C::kNV; ++u) {
-                        float kf[C::kVec];
-                        Elem<E>::to_f32(lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16),
-                                        kf);
+                        if constexpr (kFp8) {
+                            a = fmaf(dot16_e4m3(qh[u], lds128(sk + row * C::kRowBytes +
+                                                              (u * C::kG + lig) * 16)),
+                                     qinv, a);
+                        } else {
+                            float kf[C::kVec];
+                            Elem<E>::to_f32(
+                                lds128(sk + row * C::kRowBytes + (u * C::kG + lig) * 16), kf);
 #pragma unroll
-                        for (int x = 0; x < C::kVec; ++x) a = fmaf(qf[u][x], kf[x], a);
+                            for (int x = 0; x < C::kVec; ++x) a = fmaf(qf[u][x], kf[x], a);
+                        }
                     }
                 }
                 s[i] = a;
@@ -376,19 +429,62 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
                     for (int x = 0; x < C::kVec; ++x) acc[u][x] *= alpha;
+                if constexpr (kFp8) {
+                    // the tile's p v products in half precision (at most kRPG
+                    // terms per value), then added to the fp32 accumulators
+                    __half2 acch[C::kNV][C::kVec / 2];
 #pragma unroll
-                for (int i = 0; i < C::kRPG; ++i) {
-                    const int row = gi + i * C::kNG;
-                    if (row < rows) {
-                        const float pr = ex2(s[i] - mn);
-                        l += pr;
+                    for (int u = 0; u < C::kNV; ++u)
 #pragma unroll
-                        for (int u = 0; u < C::kNV; ++u) {
-                            float vf[C::kVec];
-                            Elem<E>::to_f32(
-                                lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16), vf);
+                        for (int x = 0; x < C::kVec / 2; ++x) acch[u][x] = __float2half2_rn(0.f);
 #pragma unroll
-                            for (int x = 0; x < C::kVec; ++x) acc[u][x] = fmaf(pr, vf[x], acc[u][x]);
+                    for (int i = 0; i < C::kRPG; ++i) {
+                        const int row = gi + i * C::kNG;
+                        if (row < rows) {
+                            const float pr = ex2(s[i] - mn);
+                            l += pr;
+                            const __half2 ph = __float2half2_rn(pr);
+#pragma unroll
+                            for (int u = 0; u < C::kNV; ++u) {
+                                const uint4 wv =
+                                    lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16);
+                                const uint32_t ws[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                                for (int y = 0; y < 4; ++y) {
+                                    const uint32_t lo = e4m3x2_to_f16x2(ws[y] & 0xffffu);
+                                    const uint32_t hi = e4m3x2_to_f16x2(ws[y] >> 16);
+                                    acch[u][2 * y] = __hfma2(
+                                        ph, *reinterpret_cast<const __half2*>(&lo), acch[u][2 * y]);
+                                    acch[u][2 * y + 1] =
+                                        __hfma2(ph, *reinterpret_cast<const __half2*>(&hi),
+                                                acch[u][2 * y + 1]);
+                                }
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < C::kNV; ++u)
+#pragma unroll
+                        for (int x = 0; x < C::kVec / 2; ++x) {
+                            acc[u][2 * x] += __low2float(acch[u][x]);
+                            acc[u][2 * x + 1] += __high2float(acch[u][x]);
+                        }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < C::kRPG; ++i) {
+                        const int row = gi + i * C::kNG;
+                        if (row < rows) {
+                            const float pr = ex2(s[i] - mn);
+                            l += pr;
+#pragma unroll
+                            for (int u = 0; u < C::kNV; ++u) {
+                                float vf[C::kVec];
+                                Elem<E>::to_f32(
+                                    lds128(sv + row * C::kRowBytes + (u * C::kG + lig) * 16), vf);
+#pragma unroll
+                                for (int x = 0; x < C::kVec; ++x)
+                                    acc[u][x] = fmaf(pr, vf[x], acc[u][x]);
+                            }
                         }
                     }
                 }
@@ -400,6 +496,15 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 stage = 0;
                 phase ^= 1u;
             }
+        }
+
+        if constexpr (kFp8) {
+            // the per-head value scale of the FP8 cache
+            const float vs = __ldg(p.v_scale + w.h);
+#pragma unroll
+            for (int u = 0; u < C::kNV; ++u)
+#pragma unroll
+                for (int x = 0; x < C::kVec; ++x) acc[u][x] *= vs;
         }
 
         // ---- end of piece: merge the row groups of the warp (xor butterfly)
@@ -489,10 +594,10 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
     } while (walk_next(p, ctl, w));
 }
 
-template <typename T, int D>
+template <typename TQ, typename T, int D>
 cudaError_t launch_t(int device, const PartialParams& p, cudaStream_t s) {
     using C = Cfg<T, D>;
-    auto kern = td_partial_kernel<T, D>;
+    auto kern = td_partial_kernel<TQ, T, D>;
     // the dynamic shared-memory opt-in is per device: set it once on each
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
@@ -506,13 +611,13 @@ cudaError_t launch_t(int device, const PartialParams& p, cudaStream_t s) {
     return cudaGetLastError();
 }
 
-template <typename T>
+template <typename TQ, typename T = TQ>
 cudaError_t launch_d(int device, int D, const PartialParams& p, cudaStream_t s) {
     switch (D) {
-        case 64: return launch_t<T, 64>(device, p, s);
-        case 128: return launch_t<T, 128>(device, p, s);
-        case 256: return launch_t<T, 256>(device, p, s);
-        case 512: return launch_t<T, 512>(device, p, s);
+        case 64: return launch_t<TQ, T, 64>(device, p, s);
+        case 128: return launch_t<TQ, T, 128>(device, p, s);
+        case 256: return launch_t<TQ, T, 256>(device, p, s);
+        case 512: return launch_t<TQ, T, 512>(device, p, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -539,11 +644,22 @@ cudaError_t launch_partial(int device, int dtype, int D, const PartialParams& p,
     }
 }
 
+cudaError_t launch_partial_fp8(int device, int q_dtype, int D, const PartialParams& p,
+                               cudaStream_t s) {
+    if (!p.k_scale || !p.v_scale) return cudaErrorInvalidValue;
+    switch (q_dtype) {
+        case kBF16: return launch_d<__nv_bfloat16, E4M3>(device, D, p, s);
+        case kF16: return launch_d<__half, E4M3>(device, D, p, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
 size_t partial_smem_bytes(int dtype, int D) {
     switch (dtype) {
         case kF32: return smem_d<float>(D);
         case kBF16: return smem_d<__nv_bfloat16>(D);
         case kF16: return smem_d<__half>(D);
+        case kE4M3: return smem_d<E4M3>(D);
         default: return 0;
     }
 }
