@@ -15,7 +15,9 @@ path and the fp64 oracle always see the same bits.  Recipe, per workload:
 * "peaked" workloads pick, per (b,h), ``spikes`` distinct key positions with
   ``torch.randperm`` from a CPU generator seeded with ``seed + 2`` and set
   k_j <- 8 * ||k_j|| * q/||q|| (fp32, before rounding), so those keys score far
-  above the rest.
+  above the rest (``spike_mode="aligned"``); ``spike_mode="scaled"`` takes
+  the other reading of a key spiked to eight times its norm, k_j <- 8 * k_j in
+  place, which keeps the random direction and so peaks the softmax far less.
 
 The five named workloads are the shapes the decode kernel is measured on; any
 field can be overridden (smaller N, B, H) for parity runs the oracle finishes
@@ -42,6 +44,7 @@ class Workload:
     ragged: Optional[Tuple[int, int]] = None   # inclusive [lo, hi] of N_b
     scale: float = 1.0
     spikes: int = 0
+    spike_mode: str = "aligned"  # "aligned": 8||k|| q/||q||; "scaled": 8 k in place
     seed: int = 1234
     kv_heads: int = 0           # grouped-query: key/value heads (0 = H, plain multi-head)
     prefill: bool = False       # every query row of an N-token sequence (q, k, v [B,H,N,D])
@@ -221,8 +224,13 @@ def make_inputs(w: Workload, device="cpu"):
             for h in range(H):
                 pos = torch.randperm(n_b, generator=gs)[: min(w.spikes, n_b)].to(device)
                 kj = k[b, h, pos].float()
-                qd = qf[b, h, 0] / qf[b, h, 0].norm()
-                k[b, h, pos] = (8.0 * kj.norm(dim=-1, keepdim=True) * qd).to(w.dtype)
+                if w.spike_mode == "scaled":
+                    k[b, h, pos] = (8.0 * kj).to(w.dtype)
+                elif w.spike_mode == "aligned":
+                    qd = qf[b, h, 0] / qf[b, h, 0].norm()
+                    k[b, h, pos] = (8.0 * kj.norm(dim=-1, keepdim=True) * qd).to(w.dtype)
+                else:
+                    raise ValueError("spike_mode must be 'aligned' or 'scaled'")
     slopes = alibi_slopes(H, device) if w.alibi else None
     seqlens = sl_host.to(device) if sl_host is not None else None
     return dict(q=q, k=k, v=v, slopes=slopes, seqlens=seqlens, seqlens_host=sl_host)

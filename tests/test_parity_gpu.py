@@ -288,3 +288,21 @@ def test_full_size_exact_key_counts(name):
     assert torch.allclose(got, expect, rtol=2e-7, atol=0), float((got - expect).abs().max())
     lexp = torch.log(n_b).view(B, 1, 1).expand(B, H, 1)
     assert torch.allclose(lse.double().cpu(), lexp, rtol=0, atol=4e-6)
+
+
+SPLIT_SWEEP = [16, 32, 64, 128, 256, 512, 1024]
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("mode", ["aligned", "scaled"])
+def test_peaked_1m_split_count_sweep(mode):
+    """bf16 B1 H8 D128 N=1M with 16 spiked keys per head, 16..1024 splits per
+    head: every head against the oracle at every split count (the partition
+    moves the spikes between parts, and the merge must rescale them)."""
+    w = WORKLOADS["bf16_peaked_h8_d128_n1m"].with_(spike_mode=mode)
+    inp = make_inputs(w, DEV)
+    bh = np.arange(w.B * w.H)
+    ref_o, ref_l = oracle_on(inp, bh)
+    for n_split in SPLIT_SWEEP:
+        out, lse = run_td(inp, n_split=n_split)
+        compare(out, lse, ref_o, ref_l, bh, w.dtype)
