@@ -69,7 +69,8 @@ struct KCfg {
     static constexpr int kOffP = kOffQ + kQBytes;
     static constexpr int kOffKV = ((kOffP + 2 * kPBytes) + 1023) / 1024 * 1024;
     static constexpr int kOffScratch = kOffKV + kKStages * kStageBytes;
-    // per piece parity: [group][warp quarter][head] (l, lx) and [group][head] m
+    // per piece parity: [group][head] sums of p, [head][2] output weights,
+    // [group][head] maxima
     static constexpr int kStatsFloats = 2 * (2 * 4 * GP * 2 + 2 * GP);
     static constexpr int kOffStats = kOffScratch + kKScratch * 4;
     // per group: [warp quarter][head] tile maxima
@@ -103,10 +104,6 @@ __device__ __forceinline__ void tmem_ld_x<8>(uint32_t taddr, uint32_t (&r)[8]) {
 template <>
 __device__ __forceinline__ void tmem_ld_x<16>(uint32_t taddr, uint32_t (&r)[16]) {
     tmem_ld16(taddr, r);
-}
-template <>
-__device__ __forceinline__ void tmem_ld_x<32>(uint32_t taddr, uint32_t (&r)[32]) {
-    tmem_ld32(taddr, r);
 }
 
 template <int X>
@@ -240,7 +237,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         const long long qrow0 = static_cast<long long>(w.b) * p.Hq +
                                 static_cast<long long>(w.h) * G;   // first query row
         float* stats = stats_all + (pc & 1) * (2 * 4 * GP * 2 + 2 * GP);
-        float* st_l = stats;                      // [grp][quarter][head][2]
+        float* st_l = stats;                      // [grp][head]
         float* st_m = stats + 2 * 4 * GP * 2;     // [grp][head]
 
         // Q rows of this kv head's group, K-major SW128 (rows >= G stay zero)
@@ -266,15 +263,13 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             named_bar_sync(bar_grp, kKGroup);
         }
         // per head: running max m (uniform in the group; moved when a score
-        // exceeds thr = m + 8) and this thread's sum of p over its keys.  Heads
-        // past G (padding of the MMA's N) keep m = 0 and thr = +inf: their
-        // scores are 0 (zero Q rows), their p finite and never read.
-        float m_ref[HG], thr[HG], lx[HG];
+        // exceeds m + 8) and this thread's sum of p over its keys.  Heads past G
+        // (padding of the MMA's N) keep m = 0: their scores are 0 (zero Q rows),
+        // so they never move it, and their p is finite and never read.
+        float m_ref[HG], lx[HG];
 #pragma unroll
         for (int h = 0; h < HG; ++h) {
-            const bool real = hb + h < G;
-            m_ref[h] = real ? kNegInf : 0.f;
-            thr[h] = real ? kNegInf : -kNegInf;
+            m_ref[h] = hb + h < G ? kNegInf : 0.f;
             lx[h] = 0.f;
         }
         // this thread's P^T element of head h: row hb + h, K column = key; with
@@ -292,9 +287,6 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             uint32_t sr[HG];
             tmem_ld_x<HG>(x.tmem + lane_addr + static_cast<uint32_t>(buf * NQ + hb), sr);
             tmem_wait_ld();
-            fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[buf]));
 
             if (rows < kKT && (!kSplit || grp == 0)) {
                 // keys past the piece end: p is 0 there, and 0 * NaN would poison
@@ -302,41 +294,51 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                 const int stg = static_cast<int>(t % kKStages);
                 unsigned char* vb =
                     smem + C::kOffKV + stg * C::kStageBytes + C::kAtoms * C::kKVAtom;
-                const int per_atom = (kKT - rows) * 8;  // 16-B units per atom
-                for (int u = st; u < per_atom * C::kAtoms; u += kKGroup) {
-                    const int a = u / per_atom;
-                    const int rem = u - a * per_atom;
-                    *reinterpret_cast<uint4*>(vb + a * C::kKVAtom + swz(rows + rem / 8, rem % 8)) =
-                        make_uint4(0, 0, 0, 0);
-                }
+                // 16-byte unit u: row rows + u / (8 kAtoms), atom (u / 8) % kAtoms, chunk u % 8
+                static_assert(C::kAtoms == 2, "two 64-column atoms per row");
+#pragma unroll 1
+                for (int u = st; u < (kKT - rows) * 16; u += kKGroup)
+                    *reinterpret_cast<uint4*>(vb + ((u >> 3) & 1) * C::kKVAtom +
+                                              swz(rows + (u >> 4), u & 7)) = make_uint4(0, 0, 0, 0);
                 fence_proxy_async_smem();
             }
 
-            // scores in log2 units; keys past the piece end are -inf (the
-            // select also drops whatever those K rows hold)
-            float s[HG];
+            // e = score - running max, in log2 units (one fma; the first tile of
+            // a piece, with m = -inf, gives +inf and always moves the max); keys
+            // past the piece end are -inf (the select also drops whatever those
+            // K rows hold)
+            float e[HG];
             bool need = false;
-            auto scores = [&](bool masked) {
-                const bool kvalid = key < rows;
-                const float jpos = static_cast<float>(t0 + key - w.len + 1);
+            const bool kvalid = key < rows;
+            const float jpos = static_cast<float>(t0 + key - w.len + 1);
+            auto scores = [&](bool masked, bool absolute) {
 #pragma unroll
                 for (int h = 0; h < HG; ++h) {
                     const float raw = __uint_as_float(sr[h]);
-                    float v = p.slopes ? fmaf(raw, qscale2, slope2[h] * jpos) : raw * qscale2;
+                    const float base = absolute ? 0.f : -m_ref[h];
+                    float v = p.slopes ? fmaf(raw, qscale2, fmaf(slope2[h], jpos, base))
+                                       : fmaf(raw, qscale2, base);
                     if (masked) v = kvalid ? v : kNegInf;
-                    s[h] = v;
-                    need |= v > thr[h];
+                    e[h] = v;
+                    need |= v > kKRescale;
                 }
             };
             if (rows == kKT)
-                scores(false);
+                scores(false, false);
             else
-                scores(true);
+                scores(true, false);
             if (bar_any(bar_grp, kKGroup, need)) {
-                // move the group's max to the tile max of every head
+                // move the group's max to the tile max of every head: the
+                // absolute scores again from TMEM (the S buffer is released below)
+                tmem_ld_x<HG>(x.tmem + lane_addr + static_cast<uint32_t>(buf * NQ + hb), sr);
+                tmem_wait_ld();
+                if (rows == kKT)
+                    scores(false, true);
+                else
+                    scores(true, true);
 #pragma unroll
                 for (int h = 0; h < HG; ++h) {
-                    float mx = s[h];
+                    float mx = e[h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1)
                         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -362,10 +364,10 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                     const float f = rescale(m_ref[h], mn);
                     if (hb + h < G) {
                         m_ref[h] = mn;
-                        thr[h] = mn + kKRescale;
                         lx[h] *= f;
                         if (prev >= 0) o[h] = __float_as_uint(__uint_as_float(o[h]) * f);
                     }
+                    e[h] -= m_ref[h];
                 }
                 if (prev >= 0) {
                     tmem_st_x<HG>(x.tmem + lane_addr + o_col, o);
@@ -374,6 +376,9 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                 // the maxima are read before any thread of the group can pass
                 // the next tile's reduction and overwrite them
             }
+            fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&x.s_empty[buf]));
             // the P V product of tile t - 2 read this P^T buffer
             if (t >= 2) wait_pv(t - 2);
             fence_after();
@@ -381,7 +386,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
 #pragma unroll
             for (int h = 0; h < HG; ++h) {
                 // masked keys give ex2(-inf) = 0
-                const float ev = ex2(s[h] - m_ref[h]);
+                const float ev = ex2(e[h]);
                 round_store<E>(ev, pb + h * 128 + ((kc2 ^ (h & 7)) << 4));
                 lx[h] += ev;
             }
@@ -398,102 +403,120 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             wait_pv(last_own);
             fence_after();
         }
-        // the group's sums per head: warp sums, then one partial per warp
-        float* my_l = st_l + (grp * 4 + quarter) * GP * 2;
+        // The epilogue runs once per piece, so its code is kept compact (head
+        // loops are not unrolled): it would otherwise be fetched cold into the
+        // instruction cache while the other SMs saturate L2 with K/V traffic.
+        // The group's sums of p per head, reduced through shared memory in a
+        // fixed order: [head][thread] -> kKGroup / HG partials per head -> one
+        // sum per head.  Group g uses P^T buffer g, which no P V product reads
+        // any more: in alternate mode it is the group's own buffer and its last
+        // product is complete; in split mode every product of the piece is.
+        // p is normalised by its unrounded sum (l = lx): sum_k r_k v_k / sum_k
+        // p_k differs from the exact average by at most the relative rounding of
+        // r times max |v|, as the rounded sum would.
+        constexpr int TPH = kKGroup / HG;  // partials per head
+        static_assert(kKGroup * HG * 4 <= C::kPBytes, "sum scratch");
+        float* lsum = reinterpret_cast<float*>(smem + C::kOffP + grp * C::kPBytes);
 #pragma unroll
-        for (int u = 0; u < HG; ++u) {
-            // p is normalised by its unrounded sum (l = lx): sum_k r_k v_k /
-            // sum_k p_k differs from the exact average by at most the relative
-            // rounding of r times max |v|, as the rounded sum would
-            float b = 0.f;
-            if (hb + u < G) {
-                b = lx[u];
+        for (int u = 0; u < HG; ++u) lsum[u * kKGroup + st] = lx[u];
+        if (st == 0) {
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) b += __shfl_xor_sync(0xffffffffu, b, o);
-            }
-            if (lane == 0) {
-                my_l[(hb + u) * 2 + 0] = b;
-                my_l[(hb + u) * 2 + 1] = b;
-            }
-            if (st == 0) st_m[grp * GP + hb + u] = m_ref[u];
+            for (int u = 0; u < HG; ++u) st_m[grp * GP + hb + u] = m_ref[u];
         }
-        if (kSplit) {
-            // the other group's heads: nothing from this group
-            const int ob = grp == 0 ? HG : 0;
-#pragma unroll
-            for (int u = 0; u < HG; ++u) {
-                if (lane == 0) {
-                    my_l[(ob + u) * 2 + 0] = 0.f;
-                    my_l[(ob + u) * 2 + 1] = 0.f;
-                }
-                if (st == 0) st_m[grp * GP + ob + u] = kNegInf;
+        named_bar_sync(bar_grp, kKGroup);
+        {
+            const int u = st / TPH;
+            float b = 0.f;
+#pragma unroll 1
+            for (int r = st % TPH; r < kKGroup; r += TPH) b += lsum[u * kKGroup + r];
+            named_bar_sync(bar_grp, kKGroup);
+            lsum[st] = b;  // [head][partial]
+        }
+        named_bar_sync(bar_grp, kKGroup);
+        if (st < HG) {
+            float b = 0.f;
+#pragma unroll 1
+            for (int r = 0; r < TPH; ++r) b += lsum[st * TPH + r];
+            st_l[grp * GP + hb + st] = hb + st < G ? b : 0.f;
+            if (kSplit) {
+                // the other group's heads: nothing from this group
+                const int ob = grp == 0 ? HG : 0;
+                st_l[grp * GP + ob + st] = 0.f;
+                st_m[grp * GP + ob + st] = kNegInf;
             }
         }
         fence_before();
         named_bar_sync(kBarBoth, 2 * kKGroup);
-        if (grp == 0) {
-            fence_after();
-            // a group's O^T is stale when it had no tile of this piece
-            const long long t_first = t - nt;
-            const bool has0 = kSplit || nt >= 2 || (t_first & 1) == 0;
-            const bool has1 = !kSplit && (nt >= 2 || (t_first & 1) == 1);
-            uint32_t o0[GP], o1[GP];
-            if (has0) tmem_ld_x<GP>(x.tmem + lane_addr + static_cast<uint32_t>(2 * NQ), o0);
-            if (has1) tmem_ld_x<GP>(x.tmem + lane_addr + static_cast<uint32_t>(3 * NQ), o1);
+        fence_after();
+        // a group's O^T is stale when it had no tile of this piece
+        const long long t_first = t - nt;
+        const bool has0 = kSplit || nt >= 2 || (t_first & 1) == 0;
+        const bool has1 = !kSplit && (nt >= 2 || (t_first & 1) == 1);
+        const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
+        float* const part0 = p.part + (x.c * 2 + slot) * G * (D + 3);
+        // per head, once: the merged max M and sum L of both groups, and the
+        // weights of the two O^T accumulators in the output (split mode: one
+        // accumulator, already relative to the owning group's max)
+        float* hs = stats + 8 * GP;  // [head][2]
+        if (grp == 0 && st < G) {
+            const int h = st;
+            const float m0 = st_m[h], m1 = st_m[GP + h];
+            const float M = fmaxf(m0, m1);
+            const float w0 = rescale(m0, M), w1 = rescale(m1, M);
+            const float L = w0 * st_l[h] + w1 * st_l[GP + h];
+            float a0 = kSplit ? 1.f : w0, a1 = kSplit ? 0.f : w1;
+            if (whole) {
+                a0 /= L;
+                a1 /= L;
+                if (p.lse) p.lse[qrow0 + h] = (M + log2f(L)) * kLn2;
+            } else {
+                float* rec = part0 + h * (D + 3);
+                rec[D] = M;
+                rec[D + 1] = L;
+                rec[D + 2] = L;
+            }
+            hs[2 * h] = has0 ? a0 : 0.f;
+            hs[2 * h + 1] = has1 ? a1 : 0.f;
+        }
+        named_bar_sync(kBarBoth, 2 * kKGroup);
+        // row `key` of O^T for every head, four heads per TMEM load, the two
+        // groups taking alternate blocks of four
+#pragma unroll 1
+        for (int h0 = grp * 4; h0 < G; h0 += 8) {
+            uint32_t o0[4], o1[4];
+            if (has0) tmem_ld_x<4>(x.tmem + lane_addr + static_cast<uint32_t>(2 * NQ + h0), o0);
+            if (has1) tmem_ld_x<4>(x.tmem + lane_addr + static_cast<uint32_t>(3 * NQ + h0), o1);
             tmem_wait_ld();
-            const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
 #pragma unroll
-            for (int h = 0; h < GP; ++h) {
+            for (int j = 0; j < 4; ++j) {
+                const int h = h0 + j;
                 if (h < G) {
-                    const float m0 = st_m[h], m1 = st_m[GP + h];
-                    const float M = fmaxf(m0, m1);
-                    const float w0 = rescale(m0, M), w1 = rescale(m1, M);
-                    float L = 0.f, LX = 0.f;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        L += w0 * st_l[(q * GP + h) * 2] + w1 * st_l[((4 + q) * GP + h) * 2];
-                        LX += w0 * st_l[(q * GP + h) * 2 + 1] +
-                              w1 * st_l[((4 + q) * GP + h) * 2 + 1];
-                    }
-                    // split mode: one accumulator, already relative to the
-                    // owning group's max M
-                    float v;
-                    if (kSplit) {
-                        v = __uint_as_float(o0[h]);
-                    } else {
-                        v = has0 ? __uint_as_float(o0[h]) * w0 : 0.f;
-                        if (has1) v = fmaf(w1, __uint_as_float(o1[h]), v);
-                    }
-                    const long long orow = qrow0 + h;
-                    if (whole) {
-                        p.out[orow * D + key] = v / L;
-                        if (st == 0 && p.lse) p.lse[orow] = (M + log2f(LX)) * kLn2;
-                    } else {
-                        float* rec = p.part + ((x.c * 2 + slot) * G + h) * (D + 3);
-                        rec[key] = v;
-                        if (st == 0) {
-                            rec[D] = M;
-                            rec[D + 1] = L;
-                            rec[D + 2] = LX;
-                        }
-                    }
+                    float v = has0 ? __uint_as_float(o0[j]) * hs[2 * h] : 0.f;
+                    if (has1) v = fmaf(hs[2 * h + 1], __uint_as_float(o1[j]), v);
+                    if (whole)
+                        p.out[(qrow0 + h) * D + key] = v;
+                    else
+                        part0[h * (D + 3) + key] = v;
                 }
             }
-            fence_before();
-            if (!p.fused_merge) {
-                // the CTA holding the sequence's first key describes its parts for
-                // the combine kernel (one part: already written, nothing to merge)
-                if (j0 == 0 && st == 0) {
-                    const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
-                    const long long c_lo = gpart_of(w.start, x.T, x.P);
-                    const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
-                    p.seg_desc[seg * 3 + 0] = static_cast<int>(c_lo);
-                    p.seg_desc[seg * 3 + 1] = static_cast<int>(c_hi - c_lo + 1);
-                    p.seg_desc[seg * 3 + 2] = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
-                }
-            } else if (!whole) {
-                __threadfence();
-                named_bar_sync(kBarG0, kKGroup);
+        }
+        fence_before();
+        if (!p.fused_merge) {
+            // the CTA holding the sequence's first key describes its parts for
+            // the combine kernel (one part: already written, nothing to merge)
+            if (grp == 0 && j0 == 0 && st == 0) {
+                const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
+                const long long c_lo = gpart_of(w.start, x.T, x.P);
+                const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
+                p.seg_desc[seg * 3 + 0] = static_cast<int>(c_lo);
+                p.seg_desc[seg * 3 + 1] = static_cast<int>(c_hi - c_lo + 1);
+                p.seg_desc[seg * 3 + 2] = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
+            }
+        } else if (!whole) {
+            // both groups wrote records: make them visible, then take the ticket
+            __threadfence();
+            named_bar_sync(kBarBoth, 2 * kKGroup);
+            if (grp == 0) {
                 const long long c_lo = gpart_of(w.start, x.T, x.P);
                 const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
                 const int n = static_cast<int>(c_hi - c_lo + 1);
@@ -514,8 +537,8 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                                    p.out + (qrow0 + gg) * D, p.lse ? p.lse + qrow0 + gg : nullptr);
                     }
                 }
+                named_bar_sync(kBarG0, kKGroup);
             }
-            named_bar_sync(kBarG0, kKGroup);
         }
         ++pc;
     } while (gwalk_next(p, *x.ctl, w));
@@ -577,6 +600,9 @@ __global__ void __launch_bounds__(kKThreads, 1)
     fence_before();
     __syncthreads();
     fence_after();
+    // the merge kernel that follows may be scheduled now; it waits for this
+    // grid's completion before it reads any record
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const long long T = ctl.T, x0 = ctl.x0, x1 = ctl.x1;
     const uint32_t tmem = ctl.tmem;
