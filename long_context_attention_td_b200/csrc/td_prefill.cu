@@ -55,7 +55,8 @@ struct PCfg {
     static constexpr int kOffQ = 0;
     static constexpr int kOffKV = kOffQ + kQBytes;
     static constexpr int kOffP = kOffKV + kPStages * kStageBytes;
-    static constexpr size_t kSmem = size_t(kOffP) + 2 * kPBytes + 1024;  // +align
+    static constexpr int kOffBias = kOffP + 2 * kPBytes;       // ALiBi row of a tile, x2
+    static constexpr size_t kSmem = size_t(kOffBias) + 2 * kPK * 4 + 1024;  // +align
     static_assert(D == 64 || D == 128, "D");
     static_assert(kSmem <= 232448 - 256, "shared memory");
 };
@@ -326,21 +327,51 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
             // scores in log2 units: x_c = raw_c qscale2 + slope2 (j0 + c - S + 1);
             // keys past the row's last visible key (causal) or past the
-            // sequence end are -inf
+            // sequence end are -inf.  A tile with every key visible and no bias
+            // (all but the diagonal and last tiles) takes the row max on the raw
+            // products (qscale2 > 0 keeps the order) and forms x_c - m with one
+            // fma in the exponential loop; the others build x_c first.  Maxima
+            // run as 8 independent chains (max is exact, so any order gives the
+            // same value).
             const long long j0 = t * kPK;
             const long long jmax = p.causal ? (i < p.S - 1 ? i : p.S - 1) : p.S - 1;
             const int cmax = static_cast<int>(jmax - j0 < kPK - 1 ? jmax - j0 : kPK - 1);
-            const float pos0 = static_cast<float>(j0 - p.S + 1);
-            float xs[kPK];
-            float mt = kNegInf;
+            const bool plain = p.slopes == nullptr && __all_sync(0xffffffffu, cmax == kPK - 1);
+            float mx8[8];
+            if (plain) {
 #pragma unroll
-            for (int c = 0; c < kPK; ++c) {
-                const float raw = __uint_as_float(sr[c]);
-                float x = p.slopes ? fmaf(raw, qscale2, slope2 * (pos0 + c)) : raw * qscale2;
-                x = c <= cmax ? x : kNegInf;
-                xs[c] = x;
-                mt = fmaxf(mt, x);
+                for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+#pragma unroll
+                for (int c = 8; c < kPK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
+            } else {
+                // the ALiBi row of this key tile, slope2 (j - S + 1), is the same
+                // for every query row: each thread writes one key's value
+                const float* bias = reinterpret_cast<const float*>(smem + C::kOffBias) + buf * kPK;
+                if (p.slopes) {
+                    const_cast<float*>(bias)[r] = slope2 * static_cast<float>(j0 - p.S + 1 + r);
+                    named_bar_sync(1, 4 * 32);
+                }
+                const bool masked = __any_sync(0xffffffffu, cmax < kPK - 1);
+#pragma unroll
+                for (int c = 0; c < 8; ++c) mx8[c] = kNegInf;
+#pragma unroll
+                for (int c4 = 0; c4 < kPK; c4 += 4) {
+                    const float4 b4 = p.slopes ? *reinterpret_cast<const float4*>(bias + c4)
+                                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int c = c4 + u;
+                        float x = fmaf(__uint_as_float(sr[c]), qscale2, bb[u]);
+                        if (masked) x = c <= cmax ? x : kNegInf;
+                        sr[c] = __float_as_uint(x);
+                        mx8[c & 7] = fmaxf(mx8[c & 7], x);
+                    }
+                }
             }
+            float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            if (plain) mt *= qscale2;
             // move this row's max when the tile exceeds it by more than the
             // threshold (always on the first tile)
             const bool need = mt > thr;
@@ -378,8 +409,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
                     // masked keys give ex2(-inf) = 0
-                    const float e0 = ex2(xs[cc * 8 + 2 * y] - m);
-                    const float e1 = ex2(xs[cc * 8 + 2 * y + 1] - m);
+                    const float a0 = __uint_as_float(sr[cc * 8 + 2 * y]);
+                    const float a1 = __uint_as_float(sr[cc * 8 + 2 * y + 1]);
+                    const float e0 = ex2(plain ? fmaf(a0, qscale2, -m) : a0 - m);
+                    const float e1 = ex2(plain ? fmaf(a1, qscale2, -m) : a1 - m);
                     ls[y] += e0 + e1;
                     if (kBF16)
                         asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w4[y]) : "f"(e1), "f"(e0));
