@@ -351,23 +351,29 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const_cast<float*>(bias)[r] = slope2 * static_cast<float>(j0 - p.S + 1 + r);
                     named_bar_sync(1, 4 * 32);
                 }
-                const bool masked = __any_sync(0xffffffffu, cmax < kPK - 1);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) mx8[c] = kNegInf;
+                auto build = [&](auto masked_c) {
+                    constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
-                for (int c4 = 0; c4 < kPK; c4 += 4) {
-                    const float4 b4 = p.slopes ? *reinterpret_cast<const float4*>(bias + c4)
-                                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
+                    for (int c4 = 0; c4 < kPK; c4 += 4) {
+                        const float4 b4 = p.slopes ? *reinterpret_cast<const float4*>(bias + c4)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                        const float bb[4] = {b4.x, b4.y, b4.z, b4.w};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int c = c4 + u;
-                        float x = fmaf(__uint_as_float(sr[c]), qscale2, bb[u]);
-                        if (masked) x = c <= cmax ? x : kNegInf;
-                        sr[c] = __float_as_uint(x);
-                        mx8[c & 7] = fmaxf(mx8[c & 7], x);
+                        for (int u = 0; u < 4; ++u) {
+                            const int c = c4 + u;
+                            float x = fmaf(__uint_as_float(sr[c]), qscale2, bb[u]);
+                            if (kMasked) x = c <= cmax ? x : kNegInf;
+                            sr[c] = __float_as_uint(x);
+                            mx8[c & 7] = fmaxf(mx8[c & 7], x);
+                        }
                     }
-                }
+                };
+                if (__any_sync(0xffffffffu, cmax < kPK - 1))
+                    build(std::true_type{});
+                else
+                    build(std::false_type{});
             }
             float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
@@ -403,25 +409,32 @@ __global__ void __launch_bounds__(kPThreads, 1)
             unsigned char* prow = prow0 + buf * C::kPBytes;
             // the row sum over 4 independent partials (no 128-long dependent chain)
             float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            auto exps = [&](auto plain_c) {
+                constexpr bool kPlain = decltype(plain_c)::value;
 #pragma unroll
-            for (int cc = 0; cc < kPK / 8; ++cc) {
-                uint32_t w4[4];
+                for (int cc = 0; cc < kPK / 8; ++cc) {
+                    uint32_t w4[4];
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    // masked keys give ex2(-inf) = 0
-                    const float a0 = __uint_as_float(sr[cc * 8 + 2 * y]);
-                    const float a1 = __uint_as_float(sr[cc * 8 + 2 * y + 1]);
-                    const float e0 = ex2(plain ? fmaf(a0, qscale2, -m) : a0 - m);
-                    const float e1 = ex2(plain ? fmaf(a1, qscale2, -m) : a1 - m);
-                    ls[y] += e0 + e1;
-                    if (kBF16)
-                        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w4[y]) : "f"(e1), "f"(e0));
-                    else
-                        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w4[y]) : "f"(e1), "f"(e0));
+                    for (int y = 0; y < 4; ++y) {
+                        // masked keys give ex2(-inf) = 0
+                        const float a0 = __uint_as_float(sr[cc * 8 + 2 * y]);
+                        const float a1 = __uint_as_float(sr[cc * 8 + 2 * y + 1]);
+                        const float e0 = ex2(kPlain ? fmaf(a0, qscale2, -m) : a0 - m);
+                        const float e1 = ex2(kPlain ? fmaf(a1, qscale2, -m) : a1 - m);
+                        ls[y] += e0 + e1;
+                        if (kBF16)
+                            asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w4[y]) : "f"(e1), "f"(e0));
+                        else
+                            asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w4[y]) : "f"(e1), "f"(e0));
+                    }
+                    *reinterpret_cast<uint4*>(prow + (cc >> 3) * C::kRowAtom + swz(r, cc & 7)) =
+                        make_uint4(w4[0], w4[1], w4[2], w4[3]);
                 }
-                *reinterpret_cast<uint4*>(prow + (cc >> 3) * C::kRowAtom + swz(r, cc & 7)) =
-                    make_uint4(w4[0], w4[1], w4[2], w4[3]);
-            }
+            };
+            if (plain)
+                exps(std::true_type{});
+            else
+                exps(std::false_type{});
             lx += (ls[0] + ls[1]) + (ls[2] + ls[3]);
             fence_proxy_async_smem();
             fence_before();
