@@ -40,7 +40,15 @@ using namespace dev;
 
 constexpr int kPQ = 128;             // query rows per CTA (MMA M)
 constexpr int kPK = 128;             // keys per tile (MMA N of S)
-constexpr int kPThreads = 192;       // 6 warps
+constexpr int kPThreads = 192;       // 6 warps (one softmax warpgroup)
+constexpr int kP2Threads = 384;      // 12 warps (two softmax warpgroups)
+// register split of the two-group kernel (setmaxnreg): warpgroup 0 (TMA, MMA,
+// two idle warps) drops to kRegLow, the softmax warpgroups rise to kRegHigh;
+// 4*32*kRegLow + 8*32*kRegHigh must not exceed the 384 x 168 registers the
+// block is launched with, or the increase would wait for ever
+constexpr int kRegLow = 72;
+constexpr int kRegHigh = 216;
+static_assert(4 * 32 * kRegLow + 8 * 32 * kRegHigh <= kP2Threads * 168, "register split");
 constexpr int kPStages = 2;          // K/V pipeline depth
 constexpr int kPTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256, 256 + D)
 constexpr float kPRescale = 8.f;     // log2 units
@@ -76,8 +84,11 @@ struct PCtl {
     uint32_t tmem;
 };
 
-template <typename E, int D>
-__global__ void __launch_bounds__(kPThreads, 1)
+// NG softmax groups: 1 -- one warpgroup takes every key tile; 2 -- two
+// warpgroups take alternate key tiles, each with its own running max, sum and
+// O accumulator in TMEM, merged per row at the end.
+template <typename E, int D, int NG>
+__global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
     td_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV) {
@@ -134,49 +145,63 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
     const uint32_t tmem = ctl.tmem;
     volatile int* abort_flag = &ctl.abort;
+    constexpr int kSoft0 = NG == 1 ? 2 : 4;  // first softmax warp
     const uint32_t sQ = smem_addr(smem + C::kOffQ);
     const uint32_t sKV = smem_addr(smem + C::kOffKV);
     const uint32_t sP = smem_addr(smem + C::kOffP);
     const int z = static_cast<int>(bh);
 
-    if (warp == 0) {
+    if (warp < kSoft0) {
+    // each warpgroup's register change heads its branch, so the code of the
+    // branch is compiled for that register count
+    if constexpr (NG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
+    if (warp == 0 || (NG == 2 && warp == 2)) {
         // -------------------------------------------------------- producer
+        // one warp for Q and K and (two groups) another for V, so that a K
+        // load never waits behind a V stage still held by a P V product
+        const bool doK = warp == 0;
+        const bool doV = NG == 1 || warp == 2;
         if (lane == 0) {
             bool aborted = false;
-            mbar_arrive_expect_tx(smem_addr(&q_full), C::kQBytes);
+            if (doK) {
+                mbar_arrive_expect_tx(smem_addr(&q_full), C::kQBytes);
 #pragma unroll
-            for (int a = 0; a < C::kAtoms; ++a)
-                tma_load_3d(sQ + a * C::kRowAtom, &tmQ, 64 * a, static_cast<int>(qt * kPQ), z,
-                            smem_addr(&q_full));
+                for (int a = 0; a < C::kAtoms; ++a)
+                    tma_load_3d(sQ + a * C::kRowAtom, &tmQ, 64 * a, static_cast<int>(qt * kPQ), z,
+                                smem_addr(&q_full));
+            }
             int stage = 0;
             uint32_t phase = 0;
             long long k_issued = 0, v_issued = 0;   // K / V tiles whose loads were issued
             for (long long t = 0; t < nt; ++t) {
                 const uint32_t base = sKV + stage * C::kStageBytes;
                 const int y = static_cast<int>(t * kPK);
-                if (!aborted &&
-                    !mbar_wait_bounded(smem_addr(&k_empty[stage]), phase ^ 1u, abort_flag, p.err,
-                                       TD_DEVERR_WAIT_TIMEOUT))
-                    aborted = true;
-                if (!aborted) {
-                    const uint32_t fb = smem_addr(&k_full[stage]);
-                    mbar_arrive_expect_tx(fb, C::kStageBytes / 2);
+                if (doK) {
+                    if (!aborted && !mbar_wait_bounded(smem_addr(&k_empty[stage]), phase ^ 1u,
+                                                       abort_flag, p.err, TD_DEVERR_WAIT_TIMEOUT))
+                        aborted = true;
+                    if (!aborted) {
+                        const uint32_t fb = smem_addr(&k_full[stage]);
+                        mbar_arrive_expect_tx(fb, C::kStageBytes / 2);
 #pragma unroll
-                    for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d(base + a * C::kRowAtom, &tmK, 64 * a, y, z, fb);
-                    ++k_issued;
+                        for (int a = 0; a < C::kAtoms; ++a)
+                            tma_load_3d(base + a * C::kRowAtom, &tmK, 64 * a, y, z, fb);
+                        ++k_issued;
+                    }
                 }
-                if (!aborted &&
-                    !mbar_wait_bounded(smem_addr(&v_empty[stage]), phase ^ 1u, abort_flag, p.err,
-                                       TD_DEVERR_WAIT_TIMEOUT))
-                    aborted = true;
-                if (!aborted) {
-                    const uint32_t fb = smem_addr(&v_full[stage]);
-                    mbar_arrive_expect_tx(fb, C::kStageBytes / 2);
+                if (doV) {
+                    if (!aborted && !mbar_wait_bounded(smem_addr(&v_empty[stage]), phase ^ 1u,
+                                                       abort_flag, p.err, TD_DEVERR_WAIT_TIMEOUT))
+                        aborted = true;
+                    if (!aborted) {
+                        const uint32_t fb = smem_addr(&v_full[stage]);
+                        mbar_arrive_expect_tx(fb, C::kStageBytes / 2);
 #pragma unroll
-                    for (int a = 0; a < C::kAtoms; ++a)
-                        tma_load_3d(base + (C::kAtoms + a) * C::kRowAtom, &tmV, 64 * a, y, z, fb);
-                    ++v_issued;
+                        for (int a = 0; a < C::kAtoms; ++a)
+                            tma_load_3d(base + (C::kAtoms + a) * C::kRowAtom, &tmV, 64 * a, y, z,
+                                        fb);
+                        ++v_issued;
+                    }
                 }
                 if (++stage == kPStages) {
                     stage = 0;
@@ -184,7 +209,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 }
             }
             // the CTA must not exit with copies into its shared memory in flight
-            mbar_wait_bounded(smem_addr(&q_full), 0, nullptr, p.err, TD_DEVERR_WAIT_TIMEOUT);
+            if (doK)
+                mbar_wait_bounded(smem_addr(&q_full), 0, nullptr, p.err, TD_DEVERR_WAIT_TIMEOUT);
             // tiles are issued in order, so the last K (V) load on stage s is
             // tile s + kPStages * floor((issued - 1 - s) / kPStages)
             for (int s = 0; s < kPStages; ++s) {
@@ -249,7 +275,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     const int stage = static_cast<int>(tp % kPStages);
                     const uint32_t vb = sKV + stage * C::kStageBytes + C::kAtoms * C::kRowAtom;
                     const uint32_t pb = sP + static_cast<uint32_t>((tp & 1) * C::kPBytes);
-                    const uint32_t dO = tmem + 2 * kPK;
+                    // one O accumulator per softmax group (tiles alternate)
+                    const uint32_t dO = tmem + 2 * kPK + static_cast<uint32_t>((tp % NG) * D);
 #pragma unroll
                     for (int kk = 0; kk < kPK / 16; ++kk) {
                         // P: 16 keys of every query row; V: the same 16 keys,
@@ -257,7 +284,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                         const uint64_t a = smem_desc_sw128(
                             pb + (kk >> 2) * C::kRowAtom + (kk & 3) * 32, 16, 1024);
                         const uint64_t b = smem_desc_sw128(vb + kk * 2048, C::kRowAtom, 1024);
-                        umma_f16(dO, a, b, idO, (tp > 0 || kk > 0) ? 1u : 0u);
+                        umma_f16(dO, a, b, idO, (tp >= NG || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(smem_addr(&pv_done[tp & 1]));
                     umma_commit(smem_addr(&v_empty[stage]));
@@ -295,8 +322,11 @@ __global__ void __launch_bounds__(kPThreads, 1)
                                   TD_DEVERR_WAIT_TIMEOUT);
         }
         __syncwarp();
+    }
     } else {
         // --------------------------------------------------------- softmax
+        if constexpr (NG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
+        const int g = (warp - kSoft0) >> 2;           // softmax group: tiles t % NG == g
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;            // query row of the tile (TMEM lane)
         const long long i = qt * kPQ + r;             // query index in the sequence
@@ -311,7 +341,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
         };
         float m = kNegInf, thr = kNegInf, lx = 0.f;
         unsigned char* prow0 = smem + C::kOffP;
-        for (long long t = 0; t < nt; ++t) {
+        const uint32_t o_col = static_cast<uint32_t>(2 * kPK + g * D);
+        for (long long t = g; t < nt; t += NG) {
             const int buf = static_cast<int>(t & 1);
             wait(&s_full[buf], static_cast<uint32_t>((t >> 1) & 1));
             fence_after();
@@ -346,10 +377,14 @@ __global__ void __launch_bounds__(kPThreads, 1)
             } else {
                 // the ALiBi row of this key tile, slope2 (j - S + 1), is the same
                 // for every query row: each thread writes one key's value
+                // (one buffer per tile parity; with two groups that is one per
+                // group, so the group first waits until all its warps are done
+                // with its previous tile's row)
                 const float* bias = reinterpret_cast<const float*>(smem + C::kOffBias) + buf * kPK;
                 if (p.slopes) {
+                    if (NG == 2) named_bar_sync(1 + g, 4 * 32);
                     const_cast<float*>(bias)[r] = slope2 * static_cast<float>(j0 - p.S + 1 + r);
-                    named_bar_sync(1, 4 * 32);
+                    named_bar_sync(1 + g, 4 * 32);
                 }
 #pragma unroll
                 for (int c = 0; c < 8; ++c) mx8[c] = kNegInf;
@@ -381,15 +416,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // move this row's max when the tile exceeds it by more than the
             // threshold (always on the first tile)
             const bool need = mt > thr;
-            if (__any_sync(0xffffffffu, need && t > 0)) {
-                // O holds earlier tiles: rescale this warp's rows in TMEM
-                wait(&pv_done[(t - 1) & 1], static_cast<uint32_t>(((t - 1) >> 1) & 1));
+            if (__any_sync(0xffffffffu, need && t >= NG)) {
+                // O holds this group's earlier tiles (the last one t - NG):
+                // rescale this warp's rows in TMEM
+                wait(&pv_done[(t - NG) & 1], static_cast<uint32_t>(((t - NG) >> 1) & 1));
                 fence_after();
                 const float f = need ? rescale(m, mt) : 1.f;
 #pragma unroll 1
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t o[32];
-                    const uint32_t oa = tmem + lane_addr + static_cast<uint32_t>(2 * kPK + 32 * c);
+                    const uint32_t oa = tmem + lane_addr + o_col + static_cast<uint32_t>(32 * c);
                     tmem_ld32(oa, o);
                     tmem_wait_ld();
 #pragma unroll
@@ -441,28 +477,75 @@ __global__ void __launch_bounds__(kPThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&p_full[buf]));
         }
-        // ---- the last P V product must be complete before O is read
-        if (nt > 0) wait(&pv_done[(nt - 1) & 1], static_cast<uint32_t>(((nt - 1) >> 1) & 1));
+        // ---- this group's last P V product must be complete before O is read
+        const long long last = nt > g ? g + NG * ((nt - 1 - g) / NG) : -1;
+        if (last >= 0) wait(&pv_done[last & 1], static_cast<uint32_t>((last >> 1) & 1));
         fence_after();
         // P is normalised by its unrounded sum (the rounded sum would carry
         // the same error bound)
-        const float inv = 1.f / lx;
         float* orow = p.out + (bh * p.S + i) * D;
+        if constexpr (NG == 1) {
+            const float inv = 1.f / lx;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(2 * kPK + 32 * c), o);
-            tmem_wait_ld();
-            if (i < p.S) {
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(tmem + lane_addr + o_col + static_cast<uint32_t>(32 * c), o);
+                tmem_wait_ld();
+                if (i < p.S) {
 #pragma unroll
-                for (int y = 0; y < 32; y += 4)
-                    *reinterpret_cast<float4*>(orow + 32 * c + y) =
-                        make_float4(__uint_as_float(o[y]) * inv, __uint_as_float(o[y + 1]) * inv,
-                                    __uint_as_float(o[y + 2]) * inv,
-                                    __uint_as_float(o[y + 3]) * inv);
+                    for (int y = 0; y < 32; y += 4)
+                        *reinterpret_cast<float4*>(orow + 32 * c + y) =
+                            make_float4(__uint_as_float(o[y]) * inv, __uint_as_float(o[y + 1]) * inv,
+                                        __uint_as_float(o[y + 2]) * inv,
+                                        __uint_as_float(o[y + 3]) * inv);
+                }
             }
+            if (i < p.S && p.lse) p.lse[bh * p.S + i] = (m + log2f(lx)) * kLn2;
+        } else {
+            // the two groups' (m, l) per row meet in shared memory (each group's
+            // P buffer is free once its last product is complete); the merged
+            // row is sum_g e^(m_g - M) O_g / sum_g e^(m_g - M) l_g, group g
+            // writing columns [g D/2, (g+1) D/2)
+            float* xg = reinterpret_cast<float*>(smem + C::kOffP + g * C::kPBytes);
+            xg[r] = m;
+            xg[kPQ + r] = lx;
+            fence_before();
+            named_bar_sync(3, 2 * 4 * 32);
+            fence_after();
+            const float* xa = reinterpret_cast<const float*>(smem + C::kOffP);
+            const float* xb = reinterpret_cast<const float*>(smem + C::kOffP + C::kPBytes);
+            const bool hasB = nt > 1;  // group 0 always has tile 0
+            const float mA = xa[r], mB = hasB ? xb[r] : kNegInf;
+            const float M = fmaxf(mA, mB);
+            const float wA = rescale(mA, M), wB = hasB ? rescale(mB, M) : 0.f;
+            const float L = wA * xa[kPQ + r] + (hasB ? wB * xb[kPQ + r] : 0.f);
+            const float fa = wA / L, fb = wB / L;
+#pragma unroll 1
+            for (int c = g * (D / 64); c < (g + 1) * (D / 64); ++c) {
+                uint32_t oa[32], ob[32];
+                tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(2 * kPK + 32 * c), oa);
+                if (hasB) tmem_ld32(tmem + lane_addr + static_cast<uint32_t>(2 * kPK + D + 32 * c), ob);
+                tmem_wait_ld();
+                if (i < p.S) {
+#pragma unroll
+                    for (int y = 0; y < 32; y += 4) {
+                        float4 v;
+                        v.x = __uint_as_float(oa[y]) * fa;
+                        v.y = __uint_as_float(oa[y + 1]) * fa;
+                        v.z = __uint_as_float(oa[y + 2]) * fa;
+                        v.w = __uint_as_float(oa[y + 3]) * fa;
+                        if (hasB) {
+                            v.x = fmaf(__uint_as_float(ob[y]), fb, v.x);
+                            v.y = fmaf(__uint_as_float(ob[y + 1]), fb, v.y);
+                            v.z = fmaf(__uint_as_float(ob[y + 2]), fb, v.z);
+                            v.w = fmaf(__uint_as_float(ob[y + 3]), fb, v.w);
+                        }
+                        *reinterpret_cast<float4*>(orow + 32 * c + y) = v;
+                    }
+                }
+            }
+            if (g == 0 && i < p.S && p.lse) p.lse[bh * p.S + i] = (M + log2f(L)) * kLn2;
         }
-        if (i < p.S && p.lse) p.lse[bh * p.S + i] = (m + log2f(lx)) * kLn2;
     }
 
     fence_before();
@@ -478,7 +561,8 @@ template <typename E, int D>
 cudaError_t launch_prefill_t(int device, const PrefillParams& p, const CUtensorMap& mq,
                              const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t s) {
     using C = PCfg<D>;
-    auto kern = td_prefill_kernel<E, D>;
+    constexpr int kNG = 2;
+    auto kern = td_prefill_kernel<E, D, kNG>;
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
     if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
@@ -490,7 +574,8 @@ cudaError_t launch_prefill_t(int device, const PrefillParams& p, const CUtensorM
     const long long BH = static_cast<long long>(p.B) * p.H;
     const long long nqt = (p.S + kPQ - 1) / kPQ;
     if (BH * nqt > 0x7fffffffLL) return cudaErrorInvalidValue;
-    kern<<<static_cast<unsigned>(BH * nqt), kPThreads, C::kSmem, s>>>(p, mq, mk, mv);
+    kern<<<static_cast<unsigned>(BH * nqt), kNG == 1 ? kPThreads : kP2Threads, C::kSmem, s>>>(
+        p, mq, mk, mv);
     return cudaGetLastError();
 }
 
