@@ -13,15 +13,18 @@
 // scheduled first.  Per key tile of 128 keys:
 //     S [128 q x 128 k] = Q [128 x D] . K^T       (D/16 tcgen05.mma, N = 128)
 //     O [128 q x D]    += P [128 x 128] . V       (8 tcgen05.mma, N = D)
-// with S (two buffers) and O as fp32 in TMEM, P rounded to the input type in
-// shared memory (two buffers, the A operand of P V).  Each softmax thread owns
-// one query row (its TMEM lane), so its running max and sums need no
-// cross-thread reduction; O is rescaled row by row in TMEM when a row's max
-// grows by more than 8 (log2 units).
+// with S and O as fp32 in TMEM and P rounded to the input type in shared
+// memory (the A operand of P V).  Two softmax groups take alternate key tiles,
+// each with its own S buffer, P buffer, running max and sum and O accumulator;
+// their rows are merged at the end.  Each softmax thread owns one query row
+// (its TMEM lane), so its running max and sums need no cross-thread
+// reduction; O is rescaled row by row in TMEM when a row's max grows by more
+// than 8 (log2 units).
 //
-// 6 warps: 0 TMA producer (Q once, then K and V tiles as 3-D boxes of
-// {64 columns, 128 rows, 1 sequence}, 2 stages); 1 TMEM owner and MMA issuer;
-// 2-5 softmax (warp w reads TMEM lanes 32 (w % 4) .. + 31).
+// 12 warps in three warpgroups: warpgroup 0 -- warp 0 Q and K producer, warp 2
+// V producer (3-D boxes of {64 columns, 128 rows, 1 sequence}, 2 stages),
+// warp 1 TMEM owner and MMA issuer, warp 3 idle; warpgroups 1 and 2 -- the
+// softmax groups (warp w reads TMEM lanes 32 (w % 4) .. + 31).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -40,15 +43,14 @@ using namespace dev;
 
 constexpr int kPQ = 128;             // query rows per CTA (MMA M)
 constexpr int kPK = 128;             // keys per tile (MMA N of S)
-constexpr int kPThreads = 192;       // 6 warps (one softmax warpgroup)
-constexpr int kP2Threads = 384;      // 12 warps (two softmax warpgroups)
-// register split of the two-group kernel (setmaxnreg): warpgroup 0 (TMA, MMA,
+constexpr int kPThreads = 384;       // 12 warps (two softmax warpgroups)
+// register split (setmaxnreg): warpgroup 0 (TMA, MMA,
 // two idle warps) drops to kRegLow, the softmax warpgroups rise to kRegHigh;
 // 4*32*kRegLow + 8*32*kRegHigh must not exceed the 384 x 168 registers the
 // block is launched with, or the increase would wait for ever
-constexpr int kRegLow = 72;
-constexpr int kRegHigh = 216;
-static_assert(4 * 32 * kRegLow + 8 * 32 * kRegHigh <= kP2Threads * 168, "register split");
+constexpr int kRegLow = 56;
+constexpr int kRegHigh = 224;
+static_assert(4 * 32 * kRegLow + 8 * 32 * kRegHigh <= kPThreads * 168, "register split");
 constexpr int kPStages = 2;          // K/V pipeline depth
 constexpr int kPTmemCols = 512;      // S0 [0,128) S1 [128,256) O [256, 256 + D)
 constexpr float kPRescale = 8.f;     // log2 units
@@ -84,11 +86,8 @@ struct PCtl {
     uint32_t tmem;
 };
 
-// NG softmax groups: 1 -- one warpgroup takes every key tile; 2 -- two
-// warpgroups take alternate key tiles, each with its own running max, sum and
-// O accumulator in TMEM, merged per row at the end.
-template <typename E, int D, int NG>
-__global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
+template <typename E, int D>
+__global__ void __launch_bounds__(kPThreads, 1)
     td_prefill_kernel(const PrefillParams p, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV) {
@@ -145,7 +144,7 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
 
     const uint32_t tmem = ctl.tmem;
     volatile int* abort_flag = &ctl.abort;
-    constexpr int kSoft0 = NG == 1 ? 2 : 4;  // first softmax warp
+    constexpr int kSoft0 = 4;  // first softmax warp
     const uint32_t sQ = smem_addr(smem + C::kOffQ);
     const uint32_t sKV = smem_addr(smem + C::kOffKV);
     const uint32_t sP = smem_addr(smem + C::kOffP);
@@ -154,13 +153,13 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
     if (warp < kSoft0) {
     // each warpgroup's register change heads its branch, so the code of the
     // branch is compiled for that register count
-    if constexpr (NG == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
-    if (warp == 0 || (NG == 2 && warp == 2)) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegLow));
+    if (warp == 0 || warp == 2) {
         // -------------------------------------------------------- producer
-        // one warp for Q and K and (two groups) another for V, so that a K
-        // load never waits behind a V stage still held by a P V product
+        // one warp for Q and K and another for V, so that a K load never
+        // waits behind a V stage still held by a P V product
         const bool doK = warp == 0;
-        const bool doV = NG == 1 || warp == 2;
+        const bool doV = warp == 2;
         if (lane == 0) {
             bool aborted = false;
             if (doK) {
@@ -276,7 +275,7 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
                     const uint32_t vb = sKV + stage * C::kStageBytes + C::kAtoms * C::kRowAtom;
                     const uint32_t pb = sP + static_cast<uint32_t>((tp & 1) * C::kPBytes);
                     // one O accumulator per softmax group (tiles alternate)
-                    const uint32_t dO = tmem + 2 * kPK + static_cast<uint32_t>((tp % NG) * D);
+                    const uint32_t dO = tmem + 2 * kPK + static_cast<uint32_t>((tp & 1) * D);
 #pragma unroll
                     for (int kk = 0; kk < kPK / 16; ++kk) {
                         // P: 16 keys of every query row; V: the same 16 keys,
@@ -284,7 +283,7 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
                         const uint64_t a = smem_desc_sw128(
                             pb + (kk >> 2) * C::kRowAtom + (kk & 3) * 32, 16, 1024);
                         const uint64_t b = smem_desc_sw128(vb + kk * 2048, C::kRowAtom, 1024);
-                        umma_f16(dO, a, b, idO, (tp >= NG || kk > 0) ? 1u : 0u);
+                        umma_f16(dO, a, b, idO, (tp >= 2 || kk > 0) ? 1u : 0u);
                     }
                     umma_commit(smem_addr(&pv_done[tp & 1]));
                     umma_commit(smem_addr(&v_empty[stage]));
@@ -325,8 +324,8 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
     }
     } else {
         // --------------------------------------------------------- softmax
-        if constexpr (NG == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
-        const int g = (warp - kSoft0) >> 2;           // softmax group: tiles t % NG == g
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegHigh));
+        const int g = (warp - kSoft0) >> 2;           // softmax group: tiles t % 2 == g
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;            // query row of the tile (TMEM lane)
         const long long i = qt * kPQ + r;             // query index in the sequence
@@ -342,7 +341,7 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
         float m = kNegInf, thr = kNegInf, lx = 0.f;
         unsigned char* prow0 = smem + C::kOffP;
         const uint32_t o_col = static_cast<uint32_t>(2 * kPK + g * D);
-        for (long long t = g; t < nt; t += NG) {
+        for (long long t = g; t < nt; t += 2) {
             const int buf = static_cast<int>(t & 1);
             wait(&s_full[buf], static_cast<uint32_t>((t >> 1) & 1));
             fence_after();
@@ -377,12 +376,11 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
             } else {
                 // the ALiBi row of this key tile, slope2 (j - S + 1), is the same
                 // for every query row: each thread writes one key's value
-                // (one buffer per tile parity; with two groups that is one per
-                // group, so the group first waits until all its warps are done
-                // with its previous tile's row)
+                // (one buffer per group, so the group first waits until all its
+                // warps are done with its previous tile's row)
                 const float* bias = reinterpret_cast<const float*>(smem + C::kOffBias) + buf * kPK;
                 if (p.slopes) {
-                    if (NG == 2) named_bar_sync(1 + g, 4 * 32);
+                    named_bar_sync(1 + g, 4 * 32);
                     const_cast<float*>(bias)[r] = slope2 * static_cast<float>(j0 - p.S + 1 + r);
                     named_bar_sync(1 + g, 4 * 32);
                 }
@@ -416,10 +414,10 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
             // move this row's max when the tile exceeds it by more than the
             // threshold (always on the first tile)
             const bool need = mt > thr;
-            if (__any_sync(0xffffffffu, need && t >= NG)) {
-                // O holds this group's earlier tiles (the last one t - NG):
+            if (__any_sync(0xffffffffu, need && t >= 2)) {
+                // O holds this group's earlier tiles (the last one t - 2):
                 // rescale this warp's rows in TMEM
-                wait(&pv_done[(t - NG) & 1], static_cast<uint32_t>(((t - NG) >> 1) & 1));
+                wait(&pv_done[(t - 2) & 1], static_cast<uint32_t>(((t - 2) >> 1) & 1));
                 fence_after();
                 const float f = need ? rescale(m, mt) : 1.f;
 #pragma unroll 1
@@ -478,30 +476,13 @@ __global__ void __launch_bounds__(NG == 1 ? kPThreads : kP2Threads, 1)
             if (lane == 0) mbar_arrive(smem_addr(&p_full[buf]));
         }
         // ---- this group's last P V product must be complete before O is read
-        const long long last = nt > g ? g + NG * ((nt - 1 - g) / NG) : -1;
+        const long long last = nt > g ? g + 2 * ((nt - 1 - g) / 2) : -1;
         if (last >= 0) wait(&pv_done[last & 1], static_cast<uint32_t>((last >> 1) & 1));
         fence_after();
         // P is normalised by its unrounded sum (the rounded sum would carry
         // the same error bound)
         float* orow = p.out + (bh * p.S + i) * D;
-        if constexpr (NG == 1) {
-            const float inv = 1.f / lx;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t o[32];
-                tmem_ld32(tmem + lane_addr + o_col + static_cast<uint32_t>(32 * c), o);
-                tmem_wait_ld();
-                if (i < p.S) {
-#pragma unroll
-                    for (int y = 0; y < 32; y += 4)
-                        *reinterpret_cast<float4*>(orow + 32 * c + y) =
-                            make_float4(__uint_as_float(o[y]) * inv, __uint_as_float(o[y + 1]) * inv,
-                                        __uint_as_float(o[y + 2]) * inv,
-                                        __uint_as_float(o[y + 3]) * inv);
-                }
-            }
-            if (i < p.S && p.lse) p.lse[bh * p.S + i] = (m + log2f(lx)) * kLn2;
-        } else {
+        {
             // the two groups' (m, l) per row meet in shared memory (each group's
             // P buffer is free once its last product is complete); the merged
             // row is sum_g e^(m_g - M) O_g / sum_g e^(m_g - M) l_g, group g
@@ -561,8 +542,7 @@ template <typename E, int D>
 cudaError_t launch_prefill_t(int device, const PrefillParams& p, const CUtensorMap& mq,
                              const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t s) {
     using C = PCfg<D>;
-    constexpr int kNG = 2;
-    auto kern = td_prefill_kernel<E, D, kNG>;
+    auto kern = td_prefill_kernel<E, D>;
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
     if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
@@ -574,8 +554,7 @@ cudaError_t launch_prefill_t(int device, const PrefillParams& p, const CUtensorM
     const long long BH = static_cast<long long>(p.B) * p.H;
     const long long nqt = (p.S + kPQ - 1) / kPQ;
     if (BH * nqt > 0x7fffffffLL) return cudaErrorInvalidValue;
-    kern<<<static_cast<unsigned>(BH * nqt), kNG == 1 ? kPThreads : kP2Threads, C::kSmem, s>>>(
-        p, mq, mk, mv);
+    kern<<<static_cast<unsigned>(BH * nqt), kPThreads, C::kSmem, s>>>(p, mq, mk, mv);
     return cudaGetLastError();
 }
 
