@@ -105,12 +105,20 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __shared__ PCtl ctl;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    // heaviest causal tiles first: the first wave takes the last query tile of
-    // every sequence
+    // Sequences are taken in groups of hg whose K and V together fill about
+    // 32 MB, so the query tiles in flight share key tiles in L2; inside a
+    // group the heaviest causal tiles go first (the group's last query tile
+    // of every sequence, then the one before, ...), which keeps the tail short.
     const long long BH = static_cast<long long>(p.B) * p.H;
     const long long nqt = (p.S + kPQ - 1) / kPQ;
-    const long long bh = blockIdx.x % BH;
-    const long long qt = nqt - 1 - blockIdx.x / BH;
+    const long long kv_bytes = static_cast<long long>(p.S) * D * 2 * static_cast<long long>(sizeof(E));
+    long long hg = (32ll << 20) / kv_bytes;
+    hg = hg < 1 ? 1 : (hg > BH ? BH : hg);
+    const long long grp0 = (static_cast<long long>(blockIdx.x) / (hg * nqt)) * hg;  // first sequence
+    const long long hcnt = BH - grp0 < hg ? BH - grp0 : hg;                           // its size
+    const long long idx = static_cast<long long>(blockIdx.x) - grp0 * nqt;
+    const long long bh = grp0 + idx % hcnt;
+    const long long qt = nqt - 1 - idx / hcnt;
     const long long nkt_all = (p.S + kPK - 1) / kPK;
     // key tiles this query tile reads
     const long long nt = p.causal ? (qt + 1 < nkt_all ? qt + 1 : nkt_all) : nkt_all;
