@@ -88,6 +88,7 @@ def profiled_traffic(workload, kernel="td_partial_kernel"):
     """DRAM bytes per launch of `kernel` from the committed ncu summary of this
     workload (profiles/<kernel without _kernel>_<workload>.md), or None if
     absent or taken on other sources."""
+    kernel = kernel.split(" ")[0]  # "td_partial_kernel (fp8 kv)" -> its source set
     if kernel not in KERNEL_SOURCES:
         return None
     path = os.path.join(ROOT, "profiles", "%s_%s.md" % (kernel[: -len("_kernel")], workload))
