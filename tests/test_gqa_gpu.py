@@ -76,6 +76,13 @@ def test_gqa_parts_cross_sequences(parts):
     run_and_check(w, 3, parts=parts)
 
 
+def test_gqa_merge_of_more_than_a_chunk_of_parts():
+    """1300 parts per sequence (128 keys each): the merge kernel takes the part
+    statistics in chunks of 1024 and its widest (512-thread) form."""
+    w = Workload("gqa_many", torch.bfloat16, 1, 8, 128, 1300 * 128, alibi=True, seed=800)
+    run_and_check(w, 2, parts=2 * 1300)
+
+
 def test_gqa_ragged_with_empty_sequences():
     w = Workload("gqa_r", torch.bfloat16, 5, 16, 128, 900, alibi=True, seed=600)
     run_and_check(w, 4, lens=[0, 1, 900, 333, 0])

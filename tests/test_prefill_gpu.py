@@ -97,6 +97,20 @@ def test_prefill_full_size_sampled_rows():
     check(q, k, v, sl, True, rows=rows)
 
 
+@pytest.mark.parametrize("B,H,S,D,alibi", [(3, 5, 8192, 128, True), (1, 9, 16384, 64, False)])
+def test_prefill_sequence_groups_with_a_partial_last_group(B, H, S, D, alibi):
+    """The kernel schedules sequences in groups whose K and V fill about 32 MB
+    (8 sequences here), heaviest query tiles first inside a group; with 15 and
+    9 sequences the last group is partial.  The first, last and one random row
+    of every sequence against the oracle."""
+    q, k, v, sl = inputs(B, H, S, D, torch.bfloat16, 700 + H, alibi=alibi)
+    g = np.random.default_rng(H)
+    rows = set()
+    for bh in range(B * H):
+        rows |= {bh * S, bh * S + S - 1, bh * S + int(g.integers(0, S))}
+    check(q, k, v, sl, True, rows=sorted(rows))
+
+
 def test_prefill_repeat_is_bitwise_stable_and_counted():
     q, k, v, sl = inputs(1, 2, 513, 128, torch.float16, 600, alibi=True)
     n0 = td.launch_count()
