@@ -284,6 +284,42 @@ def oracle_rate_fp8(inp, w, budget_s, min_s=0.0, threads=0):
     return bytes_once * passes / dt / 1e9, min(threads, H), desc, dt
 
 
+def sampled_parity(inp, w, out, lse, n_rows=8):
+    """The decode step's output against the fp64 oracle on sampled full-length
+    (b, h) rows of the workload: max |out - oracle| and |lse - oracle| next to
+    the bounds the parity tests hold them to (multi-head and grouped-query
+    decode; None for the other kinds)."""
+    import numpy as np
+    import oracle
+    if w.prefill or w.kv_fp8:
+        return None
+    B, H, D = w.B, w.H, w.D
+    G = H // (w.kv_heads or H)
+    lens = inp["seqlens_host"]
+    rng = np.random.default_rng(7)
+    picks = rng.choice(B * H, size=min(n_rows, B * H), replace=False)
+    rows = sorted({0, B * H - 1} | set(int(x) for x in picks))
+    q, k, v, slopes = inp["q"], inp["k"], inp["v"], inp["slopes"]
+    eo, el, used, keys = 0.0, 0.0, 0, 0
+    for r in rows:
+        b, h = divmod(r, H)
+        n_b = int(lens[b]) if lens is not None else w.N
+        if n_b == 0:
+            continue
+        qs = q[b, h].reshape(1, 1, 1, D).cpu()
+        ks = k[b, h // G, :n_b].reshape(1, 1, n_b, D).cpu()
+        vs = v[b, h // G, :n_b].reshape(1, 1, n_b, D).cpu()
+        s1 = None if slopes is None else slopes[h:h + 1].cpu()
+        ro, rl = oracle.full(qs, ks, vs, slopes=s1)
+        eo = max(eo, float(np.abs(out[b, h, 0].double().cpu().numpy() - ro[0]).max()))
+        el = max(el, abs(float(lse[b, h, 0]) - float(rl[0])))
+        used += 1
+        keys += n_b
+    bound = 1e-5 if w.dtype == torch.float32 else 2e-2
+    return {"kind": "oracle", "rows": used, "keys": keys, "max_abs_out": eo, "max_abs_lse": el,
+            "bound_out": bound, "bound_lse": 1e-4, "ok": bool(eo <= bound and el <= 1e-4)}
+
+
 def oracle_rate(inp, w, budget_s, min_s=0.0, threads=0):
     """Time the fp64 oracle on (b,h) rows of a host copy of the workload;
     returns (GB/s, threads used, description, seconds)."""
@@ -489,10 +525,15 @@ def run_ours(args):
                 "algorithmic_bytes_per_launch": int(bytes_step)}
 
     cpu = None
+    parity = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, used, desc, dt = oracle_rate(inp, w, budget_s=2.0, min_s=args.cpu_seconds)
         cpu = {"value": round(rate, 4), "unit": "GB/s", "cores": used, "kind": "oracle",
                "sample": desc, "seconds": round(dt, 2), "host_cores": os.cpu_count()}
+        try:
+            parity = sampled_parity(inp, w, out, lse)
+        except Exception as e:  # reported, never fatal to the measurement
+            parity = {"error": str(e)[:200]}
 
     if rank == 0:
         line = {
@@ -517,7 +558,7 @@ def run_ours(args):
                               "in all > 2 x 126 MB L2)" % (n_rot, bytes_step / 1e6,
                                                           n_rot * bytes_step / 1e6)),
                        "parallelism": "replicas x%d" % world},
-            "gpu_launches": int(launches), "clocks": clocks, "roofline": roofline,
+            "gpu_launches": int(launches), "clocks": clocks, "roofline": roofline, "parity": parity,
             "e2e": e2e, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
