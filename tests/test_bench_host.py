@@ -36,3 +36,47 @@ def test_sampled_parity_accepts_the_exact_result_and_flags_a_wrong_one():
 def test_sampled_parity_skips_prefill_and_fp8():
     assert bench.sampled_parity({}, WORKLOADS["prefill_bf16_h32_d128_s8k"], None, None) is None
     assert bench.sampled_parity({}, WORKLOADS["fp8kv_h32_d128_n128k"], None, None) is None
+
+
+class _Proc:
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+    def kill(self):
+        pass
+
+
+def test_clock_sampler_median_and_reasons(tmp_path):
+    """nvidia-smi rows (clocks.sm, clocks.max.sm, power.draw, event-reason
+    bits): unreadable rows are skipped, gpu_idle is not a throttle reason."""
+    p = tmp_path / "clocks.csv"
+    p.write_text("1965, 1965, 700.5, 0x0000000000000004\n"
+                 "1800, 1965, 990.1, 0x0000000000000004\n"
+                 "[N/A], 1965, 1.0, 0x0000000000000001\n"
+                 "1900, 1965, 950.0, 0x0000000000000000\n"
+                 "1500, 1965, 800.0, 0x0000000000000001\n"
+                 "truncated line\n")
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.proc, s.path, s.f = _Proc(), str(p), open(tmp_path / "sink", "w")
+    r = s.stop()
+    assert r == {"sm_mhz": 1900.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"],
+                 "samples": 4}
+
+
+def test_profiled_traffic_needs_the_current_source_hash(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "td_partial_wl.md").write_text(
+        "kernel source hash: `0123456789abcdef`\n\ndram bytes per launch: 12345\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "0123456789abcdef")
+    assert bench.profiled_traffic("wl", "td_partial_kernel") == 12345
+    # an instantiation suffix in the kernel's name maps to the same sources
+    assert bench.profiled_traffic("wl", "td_partial_kernel (fp8 kv)") == 12345
+    assert bench.profiled_traffic("other", "td_partial_kernel") is None
+    assert bench.profiled_traffic("wl", "unknown_kernel") is None
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "fedcba9876543210")
+    assert bench.profiled_traffic("wl", "td_partial_kernel") is None
