@@ -93,6 +93,11 @@ double or_decode_e4m3(uint8_t b) {
     return sign ? -v : v;
 }
 
+/* bytes per stored element of each input type */
+static size_t elem_bytes(int dtype) {
+    return dtype == OR_F64 ? 8 : dtype == OR_F32 ? 4 : 2;
+}
+
 static double load_elem(const void *base, int64_t idx, int dtype) {
     if (dtype == OR_F64) return ((const double *)base)[idx];
     if (dtype == OR_F32) return (double)((const float *)base)[idx];
@@ -297,7 +302,7 @@ static int attend_chunked(const void *q, int64_t q_off, const void *k, const voi
         const char *qb = (const char *)q;
         const char *kb = (const char *)k;
         const char *vb = (const char *)v;
-        size_t es = dtype == OR_F32 ? 4 : 2;
+        size_t es = elem_bytes(dtype);
         for (int c = 0; rc == 0 && c < w; ++c)
             rc = or_chunk_partial(qb + q_off * es, kb + kv_off * es, vb + kv_off * es,
                                   dtype, n, D, slope, starts[c], starts[c + 1],

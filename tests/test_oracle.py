@@ -281,6 +281,33 @@ def test_chunked_equals_full_every_chunk_count(mode):
         np.testing.assert_allclose(l, lse, rtol=0, atol=1e-12)
 
 
+@pytest.mark.parametrize("dtype", [torch.float64, torch.float32, torch.float16])
+@pytest.mark.parametrize("mode", ["torch_chunk", "balanced"])
+def test_chunked_equals_full_for_every_element_type_and_row(dtype, mode):
+    """The gist's claim that the chunked decode equals regular decode, on
+    every (b,h) row of a batch (so each row's q, k, v are found at their own
+    offsets) and for every element width the oracle reads (8, 4, 2 bytes),
+    with ragged lengths; the rows are also held against fp64 SDPA."""
+    B, H, N, D = 2, 3, 20, 8
+    q = _rand((B, H, 1, D), torch.float32, 111).to(dtype)
+    k = _rand((B, H, N, D), torch.float32, 112).to(dtype)
+    v = _rand((B, H, N, D), torch.float32, 113).to(dtype)
+    slopes = np.array([0.0, 0.25, 1.0], dtype=np.float32)
+    lens = torch.tensor([20, 13], dtype=torch.int32)
+    out, lse = oracle.full(q, k, v, slopes=slopes, seqlens=lens)
+    for w in range(1, 17):
+        o, l = oracle.chunked(q, k, v, w, mode, slopes=slopes, seqlens=lens)
+        np.testing.assert_allclose(o, out, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(l, lse, rtol=0, atol=1e-12)
+    for b in range(B):
+        n = int(lens[b])
+        for h in range(H):
+            ref, ref_lse = _sdpa_fp64(q[b, h, 0], k[b, h, :n], v[b, h, :n],
+                                      slope=float(slopes[h]))
+            np.testing.assert_allclose(out[b * H + h], ref, rtol=0, atol=1e-12)
+            assert abs(lse[b * H + h] - ref_lse) < 1e-12
+
+
 def test_gist_worked_case_n31_w8_d512():
     """The gist's own check: 8 ranks, 31 keys, D=512, inputs the sum of 8
     standard normal draws; Algorithm 3 must match regular decode (the page's
