@@ -2,16 +2,23 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step is one decode call over the whole workload: td_decode (the split-KV
-kernel with its fused ticket combine, one launch) for multi-head workloads, or
-td_decode_gqa (the tensor-core kernel, plus the merge kernel when sequences
-are split over many CTAs) for grouped-query ones.  Inputs are
-seeded synthetic tensors already resident in HBM; the default workload
-(bf16, B=1, H=32, D=128, N=131072) moves 2 GiB of K+V per step, far beyond the
-126 MB L2, so no flush is needed between steps (a workload whose K+V fit in
-L2 rotates over enough copies of K and V to exceed twice the L2).  Prints one JSON line on
-rank 0.  Under torchrun every rank decodes its own copy of the workload on its
-own GPU (independent problems, weak scaling, no data-path collective).
+One step is one decode call over the whole workload: td_decode /
+td_decode_varlen (the split-KV kernel with its fused ticket combine, one
+launch) for multi-head workloads, or td_decode_gqa (the tensor-core kernel,
+plus the merge kernel when sequences are split over many CTAs) for
+grouped-query ones.  Inputs are seeded synthetic tensors already resident in
+HBM; the default workload (fp16, B=64, H=16, D=64, ragged lengths U[1024,
+65536]) moves about 8.7 GB of K+V per step, far beyond the 126 MB L2, so no
+flush is needed between steps (a workload whose K+V fit in L2 rotates over
+enough copies of K and V to exceed twice the L2).  Prints one JSON line on
+rank 0.
+
+Under torchrun (N > 1 ranks) every sequence of the workload is split over the
+ranks, the gist's own multi-GPU scheme: rank r decodes chunk r of the keys of
+every sequence, the ranks exchange their partial states with one NCCL
+all-gather and each merges them (strong scaling: the total work is fixed).
+`--replicas` gives every rank its own copy of the workload instead
+(independent problems, weak scaling, no data-path collective).
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0
 only), each step a bounded sample of the same workload.
@@ -19,10 +26,13 @@ only), each step a bounded sample of the same workload.
 import argparse
 import hashlib
 import json
+import math
 import os
 import re
+import shutil
 import subprocess
 import sys
+import tempfile
 import time
 
 import torch
@@ -36,7 +46,7 @@ from long_context_attention_td_b200.workloads import (WORKLOADS, kv_bytes, kv_le
 
 METRIC = "decode attention KV GB/s and % of B200 HBM peak (1 GPU); µs per decode step"
 PREFILL_METRIC = "prefill attention TFLOP/s (4 D FLOPs per visible query-key pair; 1 GPU)"
-DEFAULT_WORKLOAD = "bf16_h32_d128_n128k"
+DEFAULT_WORKLOAD = "f16_ragged_b64_h16_d64"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
 DTYPE_NAME = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float16: "f16"}
@@ -103,6 +113,19 @@ def profiled_traffic(workload, kernel="td_partial_kernel"):
     return int(m_bytes.group(1))
 
 
+def traffic_record(workload, kernel):
+    """(traffic, where it came from) for the roofline record: the DRAM bytes
+    per launch of a committed ncu capture taken on the current kernel source,
+    or (None, why not)."""
+    t = profiled_traffic(workload, kernel)
+    base = kernel.split(" ")[0] if kernel else ""
+    name = "profiles/%s_%s.md" % (base[: -len("_kernel")], workload) if base else "-"
+    if t is None:
+        return None, "none: no ncu capture of %s on the current kernel source" % name
+    return t, ("ncu dram__bytes_read.sum + dram__bytes_write.sum from %s (kernel source hash "
+               "%s), not measured in this run" % (name, kernel_source_hash(base)))
+
+
 # ------------------------------------------------------------------ clocks
 
 _REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
@@ -126,8 +149,8 @@ class ClockSampler:
 
     def start(self):
         q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active")
-        os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
-        self.path = os.path.join(ROOT, "gpurun_out", "clocks_%d.csv" % os.getpid())
+        self.dir = tempfile.mkdtemp(prefix="td_clocks_")
+        self.path = os.path.join(self.dir, "clocks.csv")
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
@@ -138,8 +161,14 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def _cleanup(self):
+        d = getattr(self, "dir", None)
+        if d:
+            shutil.rmtree(d, ignore_errors=True)
+
     def stop(self):
         if self.proc is None:
+            self._cleanup()
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:
@@ -161,6 +190,7 @@ class ClockSampler:
             for b, n in _REASON_BITS.items():
                 if bits & b and n != "gpu_idle":
                     reasons.add(n)
+        self._cleanup()
         sm.sort()
         med = sm[len(sm) // 2] if sm else None
         return {"sm_mhz": med, "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
@@ -205,6 +235,20 @@ def barrier():
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
         dist.barrier()
+
+
+def hbm_roofline(achieved, peak, peak_kind, kernel, bytes_per_launch, traffic, traffic_src):
+    """The roofline record of an HBM-bound kernel.  `peak` is a copy rate
+    (read + write bytes of a device-to-device copy); a read-only stream can
+    run a few per cent above it, so frac may exceed 1: frac_of_nominal gives
+    the share of the 8 TB/s data-sheet bandwidth beside it."""
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
+            "peak_note": "%s device copy (read+write), the stated denominator; a read-only "
+                         "stream can exceed it" % peak_kind,
+            "frac_of_nominal": round(achieved / NOMINAL_HBM_GBS, 4),
+            "traffic": traffic, "traffic_source": traffic_src, "kernel": kernel,
+            "algorithmic_bytes_per_launch": int(bytes_per_launch)}
 
 
 # -------------------------------------------------------------- CPU oracle
@@ -482,9 +526,12 @@ def run_ours(args):
     # end to end through the host-buffer entry point (pinned host inputs)
     e2e = None
     if not args.no_e2e and not gqa and not w.kv_fp8:
-        qh = q.cpu().pin_memory()
-        kh = k.cpu().pin_memory()
-        vh = v.cpu().pin_memory()
+        def pinned(t):
+            h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            h.copy_(t)
+            return h
+
+        qh, kh, vh = pinned(q), pinned(k), pinned(v)
         sh = inp["seqlens_host"]
         slh = None if inp["slopes"] is None else inp["slopes"].cpu()
         oh = torch.empty((B, H, 1, D), dtype=torch.float32).pin_memory()
@@ -506,7 +553,10 @@ def run_ours(args):
         barrier()
         e_ms = reduce_max(e0.elapsed_time(e1), dev)
         e_bytes = reduce_sum(float(bytes_step) * e2e_steps, dev)
-        h2d = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+        # what td_decode_host copies in: q, the attended K and V rows (all of
+        # them, or the first seqlens[b] of each (b,h) of a ragged batch), the
+        # slopes and the lengths
+        h2d = qh.numel() * qh.element_size() + 2 * total_keys * D * w.elt
         h2d += 0 if slh is None else slh.numel() * 4
         h2d += 0 if sh is None else sh.numel() * 4
         d2h = oh.numel() * 4 + lh.numel() * 4
@@ -518,11 +568,9 @@ def run_ours(args):
 
     peak, peak_kind = measured_peak()
     achieved = bytes_step / (kernel_ms_max * 1e-3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "peak_kind": peak_kind,
-                "traffic": profiled_traffic(args.workload, kernel_name),
-                "kernel": kernel_name,
-                "algorithmic_bytes_per_launch": int(bytes_step)}
+    traffic, traffic_src = traffic_record(args.workload, kernel_name)
+    roofline = hbm_roofline(achieved, peak, peak_kind, kernel_name, bytes_step, traffic,
+                            traffic_src)
 
     cpu = None
     parity = None
@@ -632,6 +680,7 @@ def run_prefill(args):
     flops_all = reduce_sum(flops * args.steps, dev)
     peak, peak_kind = measured_tensor_peak()
     achieved = flops / (kernel_ms * 1e-3) / 1e12
+    traffic, tsrc = traffic_record(args.workload, kernel_name)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, used, desc, dt = oracle_rate_prefill(inp, w, budget_s=2.0, min_s=args.cpu_seconds)
@@ -653,8 +702,7 @@ def run_prefill(args):
             "gpu_launches": int(launches), "clocks": clocks,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                         "peak_kind": peak_kind, "traffic": profiled_traffic(args.workload,
-                                                                            kernel_name),
+                         "peak_kind": peak_kind, "traffic": traffic, "traffic_source": tsrc,
                          "kernel": kernel_name, "algorithmic_flops_per_launch": flops},
             "e2e": None, "cpu_baseline": cpu,
         }
@@ -666,11 +714,53 @@ def run_prefill(args):
 
 # ------------------------------------------- sequence-sharded (strong scaling)
 
+def shard_workload(inp, w, world, rank):
+    """This rank's chunk of every sequence of a materialised workload (the
+    balanced bounds of each sequence's length): a uniform workload keeps one
+    key range for all (b,h) (td_decode_shard places ALiBi terms by it); a
+    ragged one packs each sequence's chunk into [B,H,max chunk,D] with its
+    chunk lengths (no positional bias)."""
+    from long_context_attention_td_b200 import sharded
+    B, H, D, N = w.B, w.H, w.D, w.N
+    if inp["seqlens_host"] is not None:
+        if inp["slopes"] is not None:
+            raise SystemExit("a sharded ragged workload takes no ALiBi bias")
+        offs, lens = sharded.ragged_shard(inp["seqlens_host"].tolist(), world, rank, "balanced")
+        k = sharded.pack_ragged_shard(inp["k"], offs, lens)
+        v = sharded.pack_ragged_shard(inp["v"], offs, lens)
+        lens_host = torch.tensor(lens, dtype=torch.int32)
+        return {"kind": "ragged", "q": inp["q"], "k": k, "v": v,
+                "lens": lens_host.to(inp["q"].device), "lens_host": lens_host,
+                "keys": int(sum(lens)) * H, "slopes": None}
+    off, ln = sharded.shard_bounds(N, world, "balanced")[rank]
+    k = inp["k"][:, :, off:off + ln].contiguous()
+    v = inp["v"][:, :, off:off + ln].contiguous()
+    return {"kind": "uniform", "q": inp["q"], "k": k, "v": v, "off": off, "n_total": N,
+            "keys": B * H * ln, "slopes": inp["slopes"]}
+
+
+def sharded_step(ch, n_split=0, stream=None, state_fn=None, shard_fn=None, merge_fn=None):
+    """One sequence-sharded decode step of a rank on its chunk: the rank's
+    partial state, one all-gather, the merge.  The kernels may be replaced
+    by stand-ins (tests on CPU ranks)."""
+    from long_context_attention_td_b200 import sharded
+    if ch["kind"] == "ragged":
+        return sharded.decode_sharded_varlen(ch["q"], ch["k"], ch["v"], ch["lens"],
+                                             shard_lens_host=ch["lens_host"], n_split=n_split,
+                                             stream=stream, state_fn=state_fn,
+                                             merge_fn=merge_fn)
+    return sharded.decode_sharded(ch["q"], ch["k"], ch["v"], ch["off"], ch["n_total"],
+                                  slopes=ch["slopes"], n_split=n_split, stream=stream,
+                                  shard_fn=shard_fn, merge_fn=merge_fn)
+
+
 def run_sharded(args):
-    """--shard-seq: every sequence of the workload is split over the N ranks
-    (the gist's setting: rank r holds chunk r of the keys); a step is
-    td_decode_shard on the rank's chunk, one all-gather of the packed states
-    and td_merge_shards.  The total work is fixed, so this is strong scaling."""
+    """The gist's multi-GPU scheme (the default under torchrun, or --shard-seq):
+    every sequence of the workload is split over the N ranks (rank r holds
+    chunk r of its keys); a step is the rank's partial decode of its chunks
+    (td_decode_shard, or td_decode_varlen for a ragged batch), one all-gather
+    of the packed states and td_merge_shards.  The total work is fixed, so
+    this is strong scaling."""
     import long_context_attention_td_b200 as td
     from long_context_attention_td_b200 import sharded
 
@@ -680,23 +770,23 @@ def run_sharded(args):
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     w = WORKLOADS[args.workload]
-    if (w.kv_heads and w.kv_heads != w.H) or w.ragged is not None:
-        raise SystemExit("--shard-seq takes a uniform multi-head workload")
+    if (w.kv_heads and w.kv_heads != w.H) or w.prefill or w.kv_fp8:
+        raise SystemExit("the sequence-sharded step takes a multi-head decode workload")
     if args.n_keys:
         w = w.with_(N=args.n_keys)
-    off, ln = sharded.shard_bounds(w.N, world, "balanced")[rank]
-    # same seed on every rank: q is the same query everywhere; the chunk's
-    # key values do not matter for timing
-    inp = make_inputs(w.with_(N=max(ln, 1)), dev)
-    q, k, v, slopes = inp["q"], inp["k"][:, :, :ln], inp["v"][:, :, :ln], inp["slopes"]
-    k, v = k.contiguous(), v.contiguous()
+    # the same seed on every rank: every rank holds the same sequences and
+    # keeps only its chunk of them (the full tensors stay for the parity check)
+    inp = make_inputs(w, dev)
+    ch = shard_workload(inp, w, world, rank)
     stream = torch.cuda.current_stream(dev)
     n_split = w.n_split if args.n_split is None else args.n_split
-    B, H, D, N = w.B, w.H, w.D, w.N
-    bytes_all = float(2 * B * H * N * D * w.elt)
+    B, H, D = w.B, w.H, w.D
+    bytes_all = float(kv_bytes(w, inp["seqlens_host"]))
+    shard_bytes = 2 * ch["keys"] * D * w.elt
+    box = {}
 
     def step():
-        sharded.decode_sharded(q, k, v, off, N, slopes=slopes, n_split=n_split, stream=stream)
+        box["out"] = sharded_step(ch, n_split, stream)
 
     sampler = ClockSampler(dev.index).start()
     t_load0 = time.perf_counter()
@@ -716,13 +806,19 @@ def run_sharded(args):
     torch.cuda.synchronize(dev)
     barrier()
     ms_total = ev0.elapsed_time(ev1)
-    while time.perf_counter() - t_load0 < 1.2:
-        for _ in range(20):
-            step()
-        torch.cuda.synchronize(dev)
+    out, lse = box["out"]
+    out, lse = out.clone(), lse.clone()
+    # keep the GPUs loaded until the clock sampler has seen >= 1 s of load;
+    # every rank runs the same number of steps (each holds an all-gather)
+    need_s = max(0.0, 1.2 - (time.perf_counter() - t_load0))
+    n_more = int(reduce_max(float(min(20000, math.ceil(need_s / max(ms_total / args.steps * 1e-3,
+                                                                      1e-6)))), dev))
+    for _ in range(n_more):
+        step()
+    torch.cuda.synchronize(dev)
     clocks = sampler.stop()
     td.check_device_error(stream=stream)
-    # this rank's shard kernel alone, launch by launch
+    # this rank's partial-decode kernel alone, launch by launch
     n_kt = min(args.steps, 50)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(n_kt)]
@@ -730,36 +826,93 @@ def run_sharded(args):
     with torch.cuda.stream(stream):
         for a, b in evs:
             td.set_kernel_events(a, b)
-            td.decode_shard(q, k, v, off, N, state=state, slopes=slopes, n_split=n_split,
-                            stream=stream)
+            if ch["kind"] == "ragged":
+                sharded._varlen_state(ch["q"], ch["k"], ch["v"], ch["lens"], ch["lens_host"],
+                                      n_split, stream)
+            else:
+                td.decode_shard(ch["q"], ch["k"], ch["v"], ch["off"], ch["n_total"],
+                                state=state, slopes=ch["slopes"], n_split=n_split,
+                                stream=stream)
         td.set_kernel_events(None, None)
     torch.cuda.synchronize(dev)
     kernel_name = td.last_kernel()
     kernel_ms = reduce_max(sum(a.elapsed_time(b) for a, b in evs) / n_kt, dev)
     ms_max = reduce_max(ms_total, dev)
     ms_per_step = ms_max / args.steps
+
+    # end to end through the same public call: this rank's chunk copied in
+    # from pinned host memory every step, the result copied back
+    e2e = None
+    if not args.no_e2e:
+        kh = torch.empty(ch["k"].shape, dtype=ch["k"].dtype, pin_memory=True)
+        vh = torch.empty(ch["v"].shape, dtype=ch["v"].dtype, pin_memory=True)
+        qh = torch.empty(ch["q"].shape, dtype=ch["q"].dtype, pin_memory=True)
+        kh.copy_(ch["k"])
+        vh.copy_(ch["v"])
+        qh.copy_(ch["q"])
+        oh = torch.empty((B, H, 1, D), dtype=torch.float32, pin_memory=True)
+        lh = torch.empty((B, H, 1), dtype=torch.float32, pin_memory=True)
+        e2e_steps = max(3, min(args.steps, args.e2e_steps))
+
+        def e2e_step():
+            with torch.cuda.stream(stream):
+                ch["q"].copy_(qh, non_blocking=True)
+                ch["k"].copy_(kh, non_blocking=True)
+                ch["v"].copy_(vh, non_blocking=True)
+                o, l = sharded_step(ch, n_split, stream)
+                oh.copy_(o, non_blocking=True)
+                lh.copy_(l.view(B, H, 1), non_blocking=True)
+
+        e2e_step()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = reduce_max(e0.elapsed_time(e1), dev)
+        h2d = reduce_sum(float(sum(t.numel() * t.element_size() for t in (qh, kh, vh))), dev)
+        d2h = reduce_sum(float(oh.numel() * 4 + lh.numel() * 4), dev)
+        e2e = {"value": round(bytes_all * e2e_steps / (e_ms * 1e-3) / 1e9, 3), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "steps": e2e_steps, "ms_per_step": round(e_ms / e2e_steps, 4),
+               "entry_point": "sharded.decode_sharded%s (chunks copied from pinned host "
+                              "memory each step; bytes summed over ranks)"
+                              % ("_varlen" if ch["kind"] == "ragged" else "")}
+        del kh, vh, qh
+
     peak, peak_kind = measured_peak()
-    shard_bytes = 2 * B * H * ln * D * w.elt
-    achieved = shard_bytes / (kernel_ms * 1e-3) / 1e9 if ln else 0.0
+    achieved = shard_bytes / (kernel_ms * 1e-3) / 1e9 if shard_bytes else 0.0
+    parity = None
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            parity = sampled_parity(inp, w, out, lse.view(B, H, 1))
+        except Exception as e:  # reported, never fatal to the measurement
+            parity = {"error": str(e)[:200]}
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(bytes_all / (ms_per_step * 1e-3) / 1e9, 3),
             "unit": "GB/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_per_step, 6), "us_per_step": round(ms_per_step * 1e3, 3),
+            "tokens_of_kv_per_s": round(kv_lengths(w, inp["seqlens_host"]) /
+                                        (ms_per_step * 1e-3), 1),
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
             "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
-            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
-                       "B": B, "H": H, "D": D, "N": N, "alibi": w.alibi,
-                       "bytes_per_step": int(bytes_all),
-                       "l2": "no flush: K+V per rank per step %.2f GB > 126 MB L2" % (shard_bytes / 1e9),
+            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % w.N),
+                       "B": B, "H": H, "D": D, "N": w.N, "ragged": w.ragged is not None,
+                       "alibi": w.alibi, "bytes_per_step": int(bytes_all),
+                       "l2": "no flush: K+V per rank per step %.2f GB > 126 MB L2"
+                             % (shard_bytes / 1e9),
                        "parallelism": "sequence-sharded x%d" % world,
-                       "collective": "one all_gather of B*H*(D+1) fp32 per rank"},
+                       "collective": "one all_gather of B*H*(D+1) fp32 per rank (NCCL)"},
             "gpu_launches": int(launches), "clocks": clocks,
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-                         "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "peak_kind": peak_kind, "traffic": None, "kernel": kernel_name,
-                         "algorithmic_bytes_per_launch": int(shard_bytes)},
-            "e2e": None, "cpu_baseline": None,
+            "roofline": hbm_roofline(achieved, peak, peak_kind, kernel_name, shard_bytes, None,
+                                     "none: per-rank chunk, not captured"),
+            "parity": parity, "e2e": e2e, "cpu_baseline": None,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -819,14 +972,20 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--shard-seq", action="store_true",
-                    help="split every sequence over the ranks (one all-gather per step) "
-                         "instead of giving each rank its own workload")
+                    help="split every sequence over the ranks (one all-gather per step); "
+                         "the default when more than one rank runs")
+    ap.add_argument("--replicas", action="store_true",
+                    help="with more than one rank, give every rank its own copy of the "
+                         "workload (no data-path collective) instead of sharding it")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    w = WORKLOADS[args.workload]
+    shardable = not (w.prefill or w.kv_fp8 or (w.kv_heads and w.kv_heads != w.H))
     if args.impl == "reference":
         run_reference(args)
-    elif args.shard_seq:
+    elif args.shard_seq or (world > 1 and shardable and not args.replicas):
         run_sharded(args)
     elif WORKLOADS[args.workload].prefill:
         run_prefill(args)

@@ -300,19 +300,31 @@ TD_API int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, 
  *     on a B200 every D fits for B*H up to about 60,000, and D=128 up to about
  *     400,000; very large explicit n_split values may not).
  *   - The first call on a device sets up that device (looks up the array's
- *     address and zero-fills it, synchronously); make that first call before
- *     any stream capture.
+ *     address, zero-fills it and synchronises the device); make that first
+ *     call before any stream capture.
  *   - Every call on a device shares the one array and it keeps the last call's
  *     contents (tickets are left at zero by each call).  Calls that overlap on
  *     the GPU -- on different streams, or from different threads without
  *     ordering -- race on it and give wrong results: order them on one stream.
- *   - Device error bits of these calls stay in the array and are not reported
- *     by td_check_device_error.
+ *   - Device error bits of these calls are kept in the array: read and clear
+ *     them with td_check_static_error (td_check_device_error looks at the
+ *     library-owned workspace instead).
  */
 #define TD_STATIC_SCRATCH_BYTES (2u << 20)
 TD_API td_status td_decode_static(const void *q, const void *k, const void *v, float *out,
                                   float *lse, int B, int H, int64_t N, int D, int n_split,
                                   const float *alibi_slopes, td_dtype dtype, td_stream stream);
+
+/*
+ * td_check_static_error -- td_check_device_error for the fixed array of
+ * td_decode_static on the current device: waits for `stream`, reads and
+ * clears the array's error word, and returns TD_OK or TD_ERR_DEVICE with the
+ * TD_DEVERR_* bits in *bits (bits may be NULL).  After an error the whole
+ * array is zero-filled (synchronously), so the next static call starts clean.
+ * Before the first td_decode_static call on the device it only waits for
+ * `stream`.  Allocates nothing.
+ */
+TD_API td_status td_check_static_error(int *bits, td_stream stream);
 
 /* Bytes of workspace td_decode_ws needs for `parts` parts. */
 TD_API size_t td_workspace_bytes(int B, int H, int D, int64_t parts);
@@ -324,7 +336,12 @@ TD_API size_t td_workspace_bytes(int B, int H, int D, int64_t parts);
  * should be pinned for the copies to be asynchronous.  seqlens (host int32
  * [B]) may be NULL for equal lengths N.  If sync != 0 the call waits for the
  * stream before returning (out/lse are then valid); otherwise the caller
- * must synchronise `stream` before reading them.
+ * must synchronise `stream` before reading them.  Ragged batches (seqlens
+ * given) copy only the first seqlens[b] key and value rows of each (b,h),
+ * since the rows past them are never read.  The staging buffer is one per
+ * device and shared by every td_decode_host call on it: calls on different
+ * streams, or from threads without ordering, race on it -- order them on one
+ * stream.
  */
 TD_API td_status td_decode_host(const void *q, const void *k, const void *v, float *out, float *lse,
                          int B, int H, int64_t N, int D, const int32_t *seqlens,
@@ -379,6 +396,24 @@ TD_API void td_release_workspace(void);
 TD_API uint64_t td_launch_count(void);
 TD_API td_status td_set_kernel_events(void *before, void *after);
 TD_API const char *td_last_kernel(void);
+
+/*
+ * td_set_wait_test -- settings of this thread's later split-KV decode calls
+ * (td_decode, td_decode_varlen, td_decode_ws, td_decode_fp8, td_decode_shard,
+ * td_decode_static, td_decode_host) for testing the kernel's failure path.
+ * (No counterpart in the method.)  Every pipeline wait of the kernel is
+ * bounded: when a wait has not completed after wait_limit_ns nanoseconds the
+ * kernel sets TD_DEVERR_WAIT_TIMEOUT, winds down without waiting further and
+ * returns, so the context stays usable and the error is read with
+ * td_check_device_error / td_check_static_error.
+ *   wait_limit_ns   0: the default limit of 2 s; else 1000 .. 10^10.
+ *   withhold_tile   -1 (normal operation), or >= 0: the first CTA's loader
+ *                   issues its first withhold_tile tiles and then no more, so
+ *                   that CTA's next wait can only end by its limit.  The
+ *                   results of such a call are not valid.
+ * Returns TD_ERR_INVALID_ARG for values outside these ranges.
+ */
+TD_API td_status td_set_wait_test(uint64_t wait_limit_ns, int64_t withhold_tile);
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 TD_API int td_version(void);

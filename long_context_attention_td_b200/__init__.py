@@ -20,7 +20,7 @@ __all__ = [
     "TreeDecError", "lib", "library_path", "decode", "decode_varlen", "decode_ws", "combine",
     "auto_split", "plan_parts", "workspace_bytes", "decode_host", "check_device_error",
     "release_workspace", "DTYPE_CODE", "decode_gqa", "decode_gqa_ws", "plan_parts_gqa",
-    "gqa_workspace_bytes",
+    "gqa_workspace_bytes", "decode_static", "check_static_error", "set_wait_test",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -109,6 +109,12 @@ def lib():
     L.td_set_kernel_events.argtypes = [vp, vp]
     L.td_last_kernel.restype = ctypes.c_char_p
     L.td_last_kernel.argtypes = []
+    L.td_decode_static.restype = i32
+    L.td_decode_static.argtypes = [vp, vp, vp, vp, vp, i32, i32, i64, i32, i32, vp, i32, vp]
+    L.td_check_static_error.restype = i32
+    L.td_check_static_error.argtypes = [ctypes.POINTER(ctypes.c_int), vp]
+    L.td_set_wait_test.restype = i32
+    L.td_set_wait_test.argtypes = [ctypes.c_uint64, i64]
     _lib = L
     return L
 
@@ -371,6 +377,42 @@ def check_device_error(workspace=None, stream=None):
     st = lib().td_check_device_error(ws, nbytes, ctypes.byref(bits), _stream(stream))
     if st != 0:
         raise TreeDecError(st, "kernel", "error bits 0x%x" % bits.value)
+
+
+def check_static_error(stream=None):
+    """check_device_error for the fixed scratch array of decode_static."""
+    bits = ctypes.c_int(0)
+    st = lib().td_check_static_error(ctypes.byref(bits), _stream(stream))
+    if st != 0:
+        raise TreeDecError(st, "kernel (static scratch)", "error bits 0x%x" % bits.value)
+
+
+def decode_static(q, k, v, *, slopes=None, n_split=0, out=None, lse=None, stream=None):
+    """td_decode_static: decode whose scratch is a fixed array inside the
+    library, so the call allocates no device memory (out/lse may be passed in
+    for the same reason).  Calls that overlap on the GPU race on that array."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _dev_tensor(t, n)
+    B, H, N, D = _shapes(q, k, v)
+    if out is None:
+        out = torch.empty((B, H, 1, D), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    _dev_tensor(out, "out", torch.float32)
+    _dev_tensor(lse, "lse", torch.float32)
+    if slopes is not None:
+        _dev_tensor(slopes, "slopes", torch.float32)
+    st = lib().td_decode_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, D,
+                                int(n_split), _ptr(slopes), DTYPE_CODE[q.dtype], _stream(stream))
+    _check(st, "td_decode_static")
+    return out, lse
+
+
+def set_wait_test(wait_limit_ns=0, withhold_tile=-1):
+    """td_set_wait_test: limit of the split-KV kernel's pipeline waits (0: the
+    default 2 s) and the failure-path test's withheld tile (-1: off) for this
+    thread's later decode calls."""
+    _check(lib().td_set_wait_test(int(wait_limit_ns), int(withhold_tile)), "td_set_wait_test")
 
 
 def prefill(q, k, v, *, causal=True, slopes=None, out=None, lse=None, stream=None):

@@ -23,6 +23,11 @@ thread_local unsigned long long g_launches = 0;
 thread_local cudaEvent_t g_ev_before = nullptr;
 thread_local cudaEvent_t g_ev_after = nullptr;
 thread_local const char* g_last_kernel = "";
+// limit of the split-KV kernel's pipeline waits, and the failure-path test's
+// withheld tile (td_set_wait_test)
+constexpr unsigned long long kDefaultWaitNs = 2000000000ull;
+thread_local unsigned long long g_wait_ns = kDefaultWaitNs;
+thread_local long long g_withhold_tile = -1;
 std::mutex g_mu;
 
 struct DevState {
@@ -311,6 +316,8 @@ td_status decode_impl(const Req& r) {
     p.alibi_off = r.alibi_off;
     p.k_scale = r.k_scale;
     p.v_scale = r.v_scale;
+    p.wait_ns = g_wait_ns;
+    p.withhold_tile = g_withhold_tile;
     if (r.kv() == td::kE4M3)
         return cuda_status(launch_main(r.stream, "td_partial_kernel (fp8 kv)", [&] {
             return td::launch_partial_fp8(dev, r.dtype, r.D, p, r.stream);
@@ -796,6 +803,9 @@ td_status td_decode_host(const void* q, const void* k, const void* v, float* out
     const long long BH = static_cast<long long>(B) * H;
     if (!mul_fits(BH, N) || !mul_fits(BH * N, static_cast<long long>(D) * 4))
         return TD_ERR_INVALID_ARG;
+    if (seqlens)
+        for (int b = 0; b < B; ++b)
+            if (seqlens[b] < 0 || seqlens[b] > N) return TD_ERR_INVALID_ARG;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const size_t es = static_cast<size_t>(elt_size(dtype));
     const size_t qb = static_cast<size_t>(BH) * D * es;
@@ -832,8 +842,27 @@ td_status td_decode_host(const void* q, const void* k, const void* v, float* out
     }
     const cudaMemcpyKind h2d = cudaMemcpyHostToDevice;
     st = cuda_status(cudaMemcpyAsync(base + off[0], q, qb, h2d, s));
-    if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[1], k, kvb, h2d, s));
-    if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[2], v, kvb, h2d, s));
+    if (!seqlens) {
+        if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[1], k, kvb, h2d, s));
+        if (st == TD_OK) st = cuda_status(cudaMemcpyAsync(base + off[2], v, kvb, h2d, s));
+    } else {
+        // only the attended rows: for batch b, H row blocks of seqlens[b] keys
+        // at a pitch of N keys
+        const size_t row = static_cast<size_t>(D) * es;
+        const size_t pitch = static_cast<size_t>(N) * row;
+        for (int b = 0; st == TD_OK && b < B; ++b) {
+            if (seqlens[b] == 0) continue;
+            const size_t at = static_cast<size_t>(b) * H * pitch;
+            const size_t width = static_cast<size_t>(seqlens[b]) * row;
+            st = cuda_status(cudaMemcpy2DAsync(base + off[1] + at, pitch,
+                                               static_cast<const char*>(k) + at, pitch, width,
+                                               static_cast<size_t>(H), h2d, s));
+            if (st == TD_OK)
+                st = cuda_status(cudaMemcpy2DAsync(base + off[2] + at, pitch,
+                                                   static_cast<const char*>(v) + at, pitch, width,
+                                                   static_cast<size_t>(H), h2d, s));
+        }
+    }
     if (st == TD_OK && sb) st = cuda_status(cudaMemcpyAsync(base + off[5], alibi_slopes, sb, h2d, s));
     if (st == TD_OK && nb) st = cuda_status(cudaMemcpyAsync(base + off[6], seqlens, nb, h2d, s));
     if (st != TD_OK) return st;
@@ -923,6 +952,15 @@ void td_release_workspace(void) {
         s.ws_bytes = s.stage_bytes = 0;
     }
     cudaSetDevice(cur);
+}
+
+td_status td_set_wait_test(uint64_t wait_limit_ns, int64_t withhold_tile) {
+    if (wait_limit_ns != 0 && (wait_limit_ns < 1000ull || wait_limit_ns > 10000000000ull))
+        return TD_ERR_INVALID_ARG;
+    if (withhold_tile < -1) return TD_ERR_INVALID_ARG;
+    g_wait_ns = wait_limit_ns == 0 ? kDefaultWaitNs : wait_limit_ns;
+    g_withhold_tile = withhold_tile;
+    return TD_OK;
 }
 
 uint64_t td_launch_count(void) { return g_launches; }

@@ -60,18 +60,19 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 }
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up
-// (returns false, sets `code` in *err and raises *abort) after kWaitLimitNs,
-// or at once when another thread of the CTA has raised *abort.  With
-// abort == nullptr only the time limit ends the wait.
+// (returns false, sets `code` in *err and raises *abort) after limit_ns
+// nanoseconds, or at once when another thread of the CTA has raised *abort.
+// With abort == nullptr only the time limit ends the wait.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int* abort, int* err, int code) {
+                                                  volatile int* abort, int* err, int code,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 63u) == 0u) {
             if (abort != nullptr && *abort) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 atomicOr(err, code);
                 if (abort != nullptr) *abort = 1;
                 return false;

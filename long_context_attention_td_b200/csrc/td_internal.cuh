@@ -63,6 +63,9 @@ struct PartialParams {
                              // sequence is whole; a shard adds its place in the full one)
     const float* k_scale;    // FP8 K/V: per-head dequantisation scales [H] (else null)
     const float* v_scale;
+    unsigned long long wait_ns;  // limit of every pipeline wait (ns)
+    long long withhold_tile;     // >= 0: CTA 0's producer arms no stage from this tile on
+                                 // (tests the bounded-wait failure path); -1: off
 };
 
 // Grouped-query kernel (td_gqa.cu): Hq = G * Hkv query heads over Hkv kv heads.

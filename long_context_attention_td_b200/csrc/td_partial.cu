@@ -263,6 +263,9 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
         uint32_t phase = 0;
         long long issued = 0;
         bool aborted = false;
+        // the failure-path test: CTA 0 stops arming stages at this tile, so
+        // the consumers' next wait can only end by its time limit
+        const long long stop_at = c == 0 ? p.withhold_tile : -1;
         Walk w;
         if (walk_first(p, ctl, w)) {
             do {
@@ -273,8 +276,10 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
                 for (long long t0 = j0; t0 < j1; t0 += C::kTile) {
                     const long long left = j1 - t0;
                     const int rows = left < C::kTile ? static_cast<int>(left) : C::kTile;
+                    if (issued == stop_at) aborted = true;
                     if (!aborted && !mbar_wait_bounded(smem_addr(&empty_bar[stage]), phase ^ 1u,
-                                                       abort_flag, p.err, TD_DEVERR_WAIT_TIMEOUT))
+                                                       abort_flag, p.err, TD_DEVERR_WAIT_TIMEOUT,
+                                                       p.wait_ns))
                         aborted = true;
                     if (!aborted) {
                         const uint32_t bytes = static_cast<uint32_t>(rows) * C::kRowBytes;
@@ -300,7 +305,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             const long long lastTile = s + ((issued - 1 - s) / kStages) * kStages;
             const uint32_t par = static_cast<uint32_t>((lastTile / kStages) & 1);
             mbar_wait_bounded(smem_addr(&full_bar[s]), par, nullptr, p.err,
-                              TD_DEVERR_WAIT_TIMEOUT);
+                              TD_DEVERR_WAIT_TIMEOUT, p.wait_ns);
         }
         return;
     }
@@ -375,7 +380,7 @@ __global__ void __launch_bounds__(kPartialThreads, kCtasPerSm) td_partial_kernel
             const long long left = j1 - t0;
             const int rows = left < C::kTile ? static_cast<int>(left) : C::kTile;
             if (!aborted && !mbar_wait_bounded(smem_addr(&full_bar[stage]), phase, abort_flag,
-                                               p.err, TD_DEVERR_WAIT_TIMEOUT))
+                                               p.err, TD_DEVERR_WAIT_TIMEOUT, p.wait_ns))
                 aborted = true;
             const unsigned char* sk = smem + size_t(stage) * C::kStage;
             const unsigned char* sv = sk + C::kTileBytes;

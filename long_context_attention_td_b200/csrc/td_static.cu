@@ -37,7 +37,9 @@ void* g_static_ptr[kMaxDevices] = {};
 
 // Device address of the scratch on device `dev` (the current device).  The
 // first call on a device fetches it and zero-fills the array (the error word
-// and the tickets must start at zero); both are synchronous.
+// and the tickets must start at zero).  cudaMemset is ordered only on the
+// legacy default stream, which a caller's non-blocking stream does not wait
+// for, so the device is synchronised before the address is handed out.
 td_status static_scratch(int dev, void** out) {
     std::lock_guard<std::mutex> lk(g_static_mu);
     if (g_static_ptr[dev] == nullptr) {
@@ -45,8 +47,20 @@ td_status static_scratch(int dev, void** out) {
         if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || p == nullptr)
             return TD_ERR_CUDA;
         if (cudaMemset(p, 0, kScratchBytes) != cudaSuccess) return TD_ERR_CUDA;
+        if (cudaDeviceSynchronize() != cudaSuccess) return TD_ERR_CUDA;
         g_static_ptr[dev] = p;
     }
+    *out = g_static_ptr[dev];
+    return TD_OK;
+}
+
+// The scratch address of the current device if a static call has set it up,
+// else nullptr.
+td_status static_scratch_if_set(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return TD_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return TD_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_static_mu);
     *out = g_static_ptr[dev];
     return TD_OK;
 }
@@ -73,4 +87,21 @@ extern "C" td_status td_decode_static(const void* q, const void* k, const void* 
     if (st != TD_OK) return st;
     return td_decode_ws(q, k, v, out, lse, B, H, N, D, nullptr, nullptr, parts, alibi_slopes,
                         dtype, scratch, kScratchBytes, stream);
+}
+
+extern "C" td_status td_check_static_error(int* bits, td_stream stream) {
+    if (bits) *bits = 0;
+    void* scratch = nullptr;
+    const td_status st = static_scratch_if_set(&scratch);
+    if (st != TD_OK) return st;
+    if (scratch == nullptr) {
+        // no static call has run on this device: nothing can have failed,
+        // but the caller still gets the stream's own errors
+        return cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+                   ? TD_OK
+                   : TD_ERR_CUDA;
+    }
+    // the error word and the ticket/record layout of the array are those of a
+    // caller workspace of kScratchBytes
+    return td_check_device_error(scratch, kScratchBytes, bits, stream);
 }

@@ -14,7 +14,7 @@ from typing import List, Optional, Tuple
 import torch
 import torch.distributed as dist
 
-from . import decode_shard, merge_shards, state_floats
+from . import decode_shard, decode_varlen, merge_shards, state_floats
 
 
 def shard_bounds(n: int, world: int, mode: str = "torch_chunk") -> List[Tuple[int, int]]:
@@ -69,6 +69,72 @@ def decode_sharded(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor
     B, H, _, D = q.shape
     state = shard_fn(q, k_shard, v_shard, key_offset, n_total, slopes=slopes, n_split=n_split,
                      stream=stream)
+    if state.numel() != state_floats(B, H, D):
+        raise ValueError("shard state has the wrong size")
+    if alone:
+        gathered = state.view(1, -1)
+    else:
+        gathered = torch.empty((world, state.numel()), dtype=torch.float32, device=state.device)
+        _all_gather(gathered, state, group)
+    return merge_fn(gathered, B, H, D, stream=stream)
+
+
+def ragged_shard(lengths, world: int, rank: int, mode: str = "balanced"):
+    """This rank's chunk of every sequence of a ragged batch: (offsets,
+    lengths), one pair per sequence, from shard_bounds of each length."""
+    offs, lens = [], []
+    for n in lengths:
+        a, ln = shard_bounds(int(n), world, mode)[rank]
+        offs.append(a)
+        lens.append(ln)
+    return offs, lens
+
+
+def pack_ragged_shard(x: torch.Tensor, offsets, lens) -> torch.Tensor:
+    """Rows [offsets[b], offsets[b] + lens[b]) of every x[b, h] ([B,H,Nmax,D]),
+    packed into a new [B, H, max(lens), D] tensor (the rest left zero)."""
+    B, H, _, D = x.shape
+    n = max(lens) if len(lens) else 0
+    out = torch.zeros((B, H, n, D), dtype=x.dtype, device=x.device)
+    for b, (a, ln) in enumerate(zip(offsets, lens)):
+        if ln:
+            out[b, :, :ln].copy_(x[b, :, a:a + ln])
+    return out
+
+
+def _varlen_state(q, k_shard, v_shard, shard_lens, shard_lens_host, n_split=0, stream=None):
+    """td_decode_varlen on a rank's chunks, written as the packed shard state
+    (the normalised outputs, then the log-sum-exps; an empty chunk gives the
+    empty state 0 / -inf)."""
+    B, H, _, D = q.shape
+    state = torch.empty(state_floats(B, H, D), dtype=torch.float32, device=q.device)
+    if k_shard.shape[2] == 0:
+        # no keys on this rank for any sequence
+        return decode_shard(q, k_shard, v_shard, 0, 1, state=state, stream=stream)
+    decode_varlen(q, k_shard, v_shard, shard_lens, seqlens_host=shard_lens_host,
+                  n_split=n_split, out=state[: B * H * D].view(B, H, 1, D),
+                  lse=state[B * H * D:].view(B, H, 1), stream=stream)
+    return state
+
+
+def decode_sharded_varlen(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor,
+                          shard_lens: torch.Tensor, *, shard_lens_host=None, group=None,
+                          n_split: int = 0, stream=None, state_fn=None, merge_fn=None):
+    """decode_sharded for a ragged batch without a positional bias: this rank
+    holds, in k_shard/v_shard [B,H,Nmax_r,D], chunk shard_lens[b] (device
+    int32 [B]) of the keys of every sequence b (pack_ragged_shard).  The
+    attention of a chunk does not depend on where its keys sit in the
+    sequence when there is no bias, so each rank's state is a ragged decode of
+    its chunks; one all-gather and the merge finish as in decode_sharded.
+
+    state_fn(q, k, v, lens, lens_host, n_split, stream) / merge_fn default to
+    the library's kernels; a test may pass stand-ins."""
+    state_fn = state_fn or _varlen_state
+    merge_fn = merge_fn or merge_shards
+    alone = group is None and not (dist.is_available() and dist.is_initialized())
+    world = 1 if alone else dist.get_world_size(group)
+    B, H, _, D = q.shape
+    state = state_fn(q, k_shard, v_shard, shard_lens, shard_lens_host, n_split, stream)
     if state.numel() != state_floats(B, H, D):
         raise ValueError("shard state has the wrong size")
     if alone:

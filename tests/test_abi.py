@@ -179,3 +179,29 @@ def test_prefill_rejects_bad_arguments(L):
     assert L.td_prefill(p, p, p, p, p, 1, 1, 0, 128, 1, None, 1, None) == INVALID        # S
     assert L.td_prefill(odd, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID     # align
     assert L.td_prefill(None, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID
+
+
+def test_wait_test_settings_are_validated(L):
+    # limits outside 1 us .. 10 s and tiles below -1 are refused
+    assert L.td_set_wait_test(999, -1) == INVALID
+    assert L.td_set_wait_test(10_000_000_001, -1) == INVALID
+    assert L.td_set_wait_test(0, -2) == INVALID
+    assert L.td_set_wait_test(1_000_000, 3) == 0
+    assert L.td_set_wait_test(0, -1) == 0  # back to the defaults
+
+
+def test_static_entry_rejects_bad_arguments_before_setup(L):
+    p = ctypes.c_void_p(256)
+    # unsupported D / dtype and bad sizes are refused before the scratch is touched
+    assert L.td_decode_static(p, p, p, p, p, 1, 1, 16, 96, 0, None, 1, None) == UNSUPPORTED
+    assert L.td_decode_static(p, p, p, p, p, 1, 1, 16, 128, 0, None, 7, None) == UNSUPPORTED
+    assert L.td_decode_static(p, p, p, p, p, 0, 1, 16, 128, 0, None, 1, None) == INVALID
+    assert L.td_decode_static(p, p, p, p, p, 1, 1, 16, 128, -1, None, 1, None) == INVALID
+
+
+def test_host_decode_rejects_ragged_lengths_outside_the_padding(L):
+    p = ctypes.c_void_p(256)
+    lens = (ctypes.c_int32 * 2)(5, 17)   # 17 > N = 16
+    assert L.td_decode_host(p, p, p, p, p, 2, 1, 16, 128, lens, 0, None, 1, None, 0) == INVALID
+    lens = (ctypes.c_int32 * 2)(-1, 3)
+    assert L.td_decode_host(p, p, p, p, p, 2, 1, 16, 128, lens, 0, None, 1, None, 0) == INVALID

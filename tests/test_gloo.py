@@ -218,3 +218,68 @@ def test_shard_bounds_match_the_oracle_chunking(n, world):
         starts = oracle.chunk_bounds(n, world, mode)
         got = sharded.shard_bounds(n, world, mode)
         assert [(a, b - a) for a, b in zip(starts[:-1], starts[1:])] == got
+
+
+def _oracle_varlen_state(q, k_s, v_s, lens, lens_host, n_split=0, stream=None):
+    """The ragged shard state (td_decode_varlen on a rank's chunks) computed
+    by the oracle: a chunk of length 0 gives the empty state (0, -inf)."""
+    import oracle
+    B, H, _, D = q.shape
+    if k_s.shape[2] == 0:
+        return torch.cat([torch.zeros(B * H * D), torch.full((B * H,), -math.inf)]).float()
+    o, l = oracle.full(q, k_s, v_s, seqlens=lens_host)
+    return torch.from_numpy(np.concatenate([o.ravel(), l])).to(torch.float32)
+
+
+def _bench_sharded(rank, world, port, name, kw, result):
+    import bench
+    from long_context_attention_td_b200.workloads import WORKLOADS, make_inputs
+    _init(rank, world, port)
+    try:
+        w = WORKLOADS[name].with_(**kw)
+        inp = make_inputs(w, "cpu")
+        ch = bench.shard_workload(inp, w, world, rank)
+        out, lse = bench.sharded_step(ch, state_fn=_oracle_varlen_state,
+                                      shard_fn=_oracle_shard_state, merge_fn=_oracle_merge)
+        result.put((rank, ch["keys"], np.asarray(out).tolist(), np.asarray(lse).tolist()))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world,name,kw", [
+    (2, "f16_ragged_b64_h16_d64", dict(B=5, H=2, N=40, ragged=(1, 40))),
+    (3, "f16_ragged_b64_h16_d64", dict(B=4, H=3, N=9, ragged=(0, 9))),
+    (2, "bf16_alibi_b8_h32_d128_n32k", dict(B=2, H=3, N=33)),
+    (3, "bf16_h32_d128_n128k", dict(H=2, N=50)),
+])
+def test_bench_sharded_step_on_cpu_ranks(world, name, kw):
+    """bench.py's multi-GPU step (each rank takes its chunk of every sequence
+    with shard_workload, then decodes it, all-gathers the states and merges)
+    on gloo ranks, with the oracle standing in for the kernels: every rank
+    ends with the plain definition over the whole workload, and the chunks
+    cover every attended key exactly once."""
+    import oracle
+    from long_context_attention_td_b200.workloads import WORKLOADS, kv_lengths, make_inputs
+    ctx = mp.get_context("spawn")
+    result = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bench_sharded, args=(r, world, port, name, kw, result))
+             for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [result.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    w = WORKLOADS[name].with_(**kw)
+    inp = make_inputs(w, "cpu")
+    s = None if inp["slopes"] is None else inp["slopes"].numpy()
+    ref, ref_l = oracle.full(inp["q"], inp["k"], inp["v"], slopes=s, seqlens=inp["seqlens_host"])
+    assert sum(g[1] for g in got) == kv_lengths(w, inp["seqlens_host"])
+    fin = np.isfinite(ref_l)
+    for _, _, out, lse in got:
+        out = np.array(out).reshape(ref.shape)
+        lse = np.array(lse).reshape(-1)
+        np.testing.assert_allclose(out, ref, rtol=0, atol=2e-6)
+        np.testing.assert_allclose(lse[fin], ref_l[fin], rtol=0, atol=2e-6)
+        assert np.all(lse[~fin] == -np.inf)
