@@ -263,9 +263,12 @@ TD_API td_status td_prefill(const void *q, const void *k, const void *v, float *
 /*
  * td_auto_split -- the split heuristic: the number of parts (CTAs) for T =
  * B*H*N attended keys on a GPU with num_sms SMs: enough to fill every SM with
- * as many CTAs as fit at once, but no part smaller than 64 KiB of K+V and
- * never more parts than keys.  Pure host arithmetic (no GPU needed).
- * Returns -1 on invalid arguments.
+ * as many CTAs as fit at once, but no part smaller than 64 KiB of K+V, no more
+ * than floor(sqrt(0.62 * N * element bytes)) parts per sequence (beyond that
+ * the merge of a sequence's parts by its last CTA costs more than the shorter
+ * parts save: about 100 parts for N = 4096 fp32 keys), and never more parts
+ * than keys.  Pure host arithmetic (no GPU needed).  Returns -1 on invalid
+ * arguments.
  */
 TD_API int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int num_sms);
 

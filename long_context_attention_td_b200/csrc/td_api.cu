@@ -124,7 +124,16 @@ size_t ws_bytes_for(long long BH, int D, long long parts) {
            static_cast<size_t>(parts) * 2 * static_cast<size_t>(D + 2) * sizeof(float);
 }
 
-long long auto_parts(long long T, int D, int dtype, int num_sms) {
+// The split heuristic over T attended keys of BH sequences: fill every SM with
+// as many CTAs as fit at once, no part below kMinPartBytes of K+V, and no more
+// parts per sequence than keep the merge cheap.  The last CTA of a sequence
+// reads all of its n part records ((D+2) floats each) at about the rate one
+// CTA streams K/V (measured ~62 vs ~50 GB/s on B200), so a part count n per
+// sequence of average length L costs ~ 2 L D elt / n + 4 D n / 1.24 bytes of
+// one CTA's time, smallest at n = sqrt(0.62 L elt): ~100 for 4096 fp32 keys,
+// ~400 for 128K bf16 keys -- a cap that only shows when few, short sequences
+// would otherwise be cut into hundreds of parts.
+long long auto_parts(long long T, long long BH, int D, int dtype, int num_sms) {
     if (T <= 0) return 1;
     const long long fill = static_cast<long long>(num_sms) * td::partial_ctas_per_sm(dtype, D);
     const long long bytes_per_key = 2LL * D * elt_size(dtype);
@@ -133,6 +142,12 @@ long long auto_parts(long long T, int D, int dtype, int num_sms) {
                                  : 1);
     if (by_size < 1) by_size = 1;
     long long P = fill < by_size ? fill : by_size;
+    if (BH > 0) {
+        const double L = static_cast<double>(T) / static_cast<double>(BH);
+        long long per_seq = static_cast<long long>(std::sqrt(0.62 * L * elt_size(dtype)));
+        if (per_seq < 1) per_seq = 1;
+        if (mul_fits(BH, per_seq) && P > BH * per_seq) P = BH * per_seq;
+    }
     if (P > T) P = T;
     return P < 1 ? 1 : P;
 }
@@ -276,7 +291,9 @@ long long plan_parts(const Req& r, int num_sms) {
     const long long bound = static_cast<long long>(r.B) * r.H * r.N;
     const long long known = known_keys(r);
     const long long T = known >= 0 ? known : bound;
-    long long P = r.parts > 0 ? r.parts : auto_parts(T, r.D, r.kv(), num_sms);
+    long long P = r.parts > 0 ? r.parts
+                              : auto_parts(T, static_cast<long long>(r.B) * r.H, r.D, r.kv(),
+                                           num_sms);
     const long long cap = T > 0 ? T : 1;
     if (P > cap) P = cap;
     if (P > 0x7fffffffLL) P = 0x7fffffffLL;
@@ -346,9 +363,10 @@ size_t gqa_ws_bytes_for(long long BHkv, int G, int D, long long parts) {
                static_cast<size_t>(D + 3) * sizeof(float);
 }
 
-long long gqa_auto_parts(long long T, int D, int num_sms) {
+long long gqa_auto_parts(long long T, int D, int G, int num_sms) {
     if (T <= 0) return 1;
-    const long long fill = static_cast<long long>(num_sms) * kGqaCtasPerSm;
+    const int per_sm = td::gqa_keys_path(D, G) ? td::gqa_keys_ctas_per_sm(D, G) : kGqaCtasPerSm;
+    const long long fill = static_cast<long long>(num_sms) * per_sm;
     const long long bytes_per_key = 2LL * D * 2;
     long long by_size = T / (td::kMinPartBytes / bytes_per_key);
     if (by_size < 1) by_size = 1;
@@ -414,7 +432,7 @@ long long gqa_plan(const GqaReq& r, int num_sms) {
         const long long per = (!r.seqlens && r.n_split > r.N) ? r.N : r.n_split;
         P = BHkv * per;
     }
-    if (P == 0) P = gqa_auto_parts(T, r.D, num_sms);
+    if (P == 0) P = gqa_auto_parts(T, r.D, r.Hq / r.Hkv, num_sms);
     const long long cap = T > 0 ? T : 1;
     if (P > cap) P = cap;
     if (P > 0x7fffffffLL) P = 0x7fffffffLL;
@@ -504,8 +522,8 @@ td_status gqa_impl(const GqaReq& r) {
     st = cuda_status(launch_main(r.stream, keys_path ? "td_gqa_keys_kernel" : "td_gqa_kernel",
                                  [&] {
                                      return keys_path
-                                                ? td::launch_gqa_keys(dev, r.dtype, p, mk, mv,
-                                                                      r.stream)
+                                                ? td::launch_gqa_keys(dev, r.dtype, r.D, p, mk,
+                                                                      mv, r.stream)
                                                 : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv,
                                                                  r.stream);
                                  }));
@@ -627,7 +645,7 @@ int64_t td_plan_parts_gqa(int B, int Hq, int Hkv, int64_t Nmax, int D, td_dtype 
     if (total_keys >= 0) {
         // ragged: size from the given key count
         long long T = total_keys;
-        long long P = n_split > 0 ? BHkv * n_split : gqa_auto_parts(T, D, sms);
+        long long P = n_split > 0 ? BHkv * n_split : gqa_auto_parts(T, D, Hq / Hkv, sms);
         const long long cap = T > 0 ? T : 1;
         if (P > cap) P = cap;
         return P < 1 ? 1 : P;
@@ -764,7 +782,7 @@ int64_t td_auto_split(int B, int H, int64_t N, int D, td_dtype dtype, int num_sm
     if (B < 1 || H < 1 || N < 1 || num_sms < 1 || !dtype_ok(dtype) || !d_ok(D)) return -1;
     const long long BH = static_cast<long long>(B) * H;
     if (!mul_fits(BH, N)) return -1;
-    return auto_parts(BH * N, D, dtype, num_sms);
+    return auto_parts(BH * N, BH, D, dtype, num_sms);
 }
 
 int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, int n_split,
@@ -782,7 +800,7 @@ int64_t td_plan_parts(int B, int H, int64_t Nmax, int D, td_dtype dtype, int n_s
         const long long per = n_split < Nmax ? n_split : Nmax;
         parts = total_keys < 0 ? BH * per : BH * n_split;
     }
-    long long P = parts > 0 ? parts : auto_parts(T, D, dtype, sms);
+    long long P = parts > 0 ? parts : auto_parts(T, BH, D, dtype, sms);
     const long long cap = T > 0 ? T : 1;
     if (P > cap) P = cap;
     return P < 1 ? 1 : P;

@@ -264,7 +264,7 @@ __device__ void tree_merge(const Acc& acc, int n, int D, int t, int nthreads, fl
             if (sl < SL) {
                 const int d0 = dd, d1 = DL + dd;
                 const bool two = passes > 1 && d1 < D;
-                constexpr int kBatch = 8;  // independent record loads in flight per thread
+                constexpr int kBatch = 16;  // independent record loads in flight per thread
                 int i = sl;
 #pragma unroll 1
                 for (; i + (kBatch - 1) * SL < cnt; i += kBatch * SL) {

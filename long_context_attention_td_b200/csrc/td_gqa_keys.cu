@@ -9,7 +9,7 @@
 //     O^T [D x NQ]        += V^T [D x 128] . P^T [128 x NQ]
 // where the NQ columns are the group's query heads (G padded to 16 or 32).
 // One tcgen05.mma (K = 16) covers 16 columns of D in the first product and 16
-// keys in the second, so a tile takes 2 x 8 instructions, and the operands
+// keys in the second, so a tile takes D/16 + 8 instructions, and the operands
 // the tensor core reads from shared memory are the K and V tiles once plus a
 // small Q or P block.  With the query heads on M instead, the same 128 keys
 // take 24 instructions and re-read the 128-row Q block for every one of them.
@@ -20,14 +20,20 @@
 // exceeds it by more than 8 (log2 units), which one barrier-reduction per
 // tile decides, and O^T in TMEM is rescaled then.
 //
+// For D = 64 the P V product still runs with M = 128: the second 64-row half
+// of its A operand is the stage's K tile, so rows 64-127 of O^T hold values
+// that are never read, and the TMEM layout of O^T (row r in lane r) is the one
+// the D = 128 kernel uses.
+//
 // One CTA per SM, 10 warps:
 //   warp 0      TMA producer: K and V tiles of 128 keys as 2-D boxes of
-//               {64 columns, 128 rows} with 128-byte swizzle, 3 stages;
+//               {64 columns, 128 rows} with 128-byte swizzle, 3 stages of
+//               64 KB (D = 128) or 6 stages of 32 KB (D = 64);
 //   warp 1      owns TMEM (S0, S1, O0, O1: NQ columns each) and issues the
 //               MMAs from one lane, signalling completion with tcgen05.commit;
 //   warps 2-5   softmax group 0 (even tiles), warps 6-9 group 1 (odd tiles);
 //               warp w reads TMEM lanes 32 (w % 4) .. + 31.
-// Used for D = 128 and G <= 32; td_gqa covers the other shapes.
+// Used for D = 64 or 128 and G <= 32; td_gqa covers the other shapes.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -45,8 +51,7 @@ namespace {
 using namespace dev;
 
 constexpr int kKT = 128;              // keys per tile (MMA M of S^T)
-constexpr int kKD = 128;              // head dimension (MMA M of O^T)
-constexpr int kKStages = 3;           // K/V pipeline depth (64 KB per stage)
+constexpr int kKMO = 128;             // MMA M of O^T (D rows, padded to 128 for D = 64)
 constexpr int kKThreads = 320;        // 10 warps
 constexpr int kKGroup = 128;          // threads of one softmax warpgroup
 constexpr int kKScratch = 512;        // floats of tree_merge scratch (>= 128)
@@ -55,20 +60,29 @@ constexpr int kBarG0 = 1;             // named barrier: softmax group 0
 constexpr int kBarBoth = 2;           // named barrier: both softmax groups
 constexpr int kBarG1 = 3;             // named barrier: softmax group 1
 
-template <int GP>
+template <int GP, int D>
 struct KCfg {
     static constexpr int NQ = GP < 16 ? 16 : GP;      // MMA N
-    static constexpr int kAtoms = kKD / 64;            // 64-column swizzle atoms of D
+    static constexpr int kAtoms = D / 64;              // 64-column swizzle atoms of D
+    // CTAs per SM: two for D = 64 up to 16 heads per group (their 32 KB tiles
+    // leave room for two CTAs of 3 stages each), else one
+    static constexpr int kCtasPerSm = (D == 64 && GP <= 16) ? 2 : 1;
+    static constexpr int kStages = D == 128 ? 3 : (kCtasPerSm == 2 ? 3 : 6);  // K/V depth
     static constexpr int kQAtom = NQ * 128;            // NQ rows x 64 columns
     static constexpr int kQBytes = kAtoms * kQAtom;
     static constexpr int kPAtom = NQ * 128;            // NQ rows x 64 keys
     static constexpr int kPBytes = (kKT / 64) * kPAtom;  // one P^T buffer
     static constexpr int kKVAtom = kKT * 128;          // 128 keys x 64 columns
-    static constexpr int kStageBytes = 2 * kAtoms * kKVAtom;  // K atoms, then V atoms
+    static constexpr int kStageBytes = 2 * kAtoms * kKVAtom;
+    // inside a stage: D = 128, the K atoms then the V atoms; D = 64, the V atom
+    // then the K atom, so the P V product's rows 64-127 (its A operand's second
+    // 64-row half, kKVAtom past the V atom) read this stage's K tile
+    static constexpr int kOffKAtoms = D == 128 ? 0 : kKVAtom;
+    static constexpr int kOffVAtoms = D == 128 ? kAtoms * kKVAtom : 0;
     static constexpr int kOffQ = 0;
     static constexpr int kOffP = kOffQ + kQBytes;
     static constexpr int kOffKV = ((kOffP + 2 * kPBytes) + 1023) / 1024 * 1024;
-    static constexpr int kOffScratch = kOffKV + kKStages * kStageBytes;
+    static constexpr int kOffScratch = kOffKV + kStages * kStageBytes;
     // per piece parity: [group][head] sums of p, [head][2] output weights,
     // [group][head] maxima
     static constexpr int kStatsFloats = 2 * (2 * 4 * GP * 2 + 2 * GP);
@@ -81,7 +95,9 @@ struct KCfg {
     static constexpr size_t kSmem = size_t(kOffSlopes) + 2 * GP * 4 + 1024;  // +align
     static constexpr int kTmemCols = 4 * NQ < 32 ? 32 : 4 * NQ;
     static_assert(GP == 4 || GP == 8 || GP == 16 || GP == 32, "GP");
+    static_assert(D == 64 || D == 128, "D");
     static_assert(kSmem <= 232448 - 512, "shared memory");
+    static_assert(kCtasPerSm * (kSmem + 1024) <= 233472, "shared memory of the CTAs of an SM");
 };
 
 // ----------------------------------------------------------- TMEM access
@@ -193,11 +209,10 @@ struct KCtx {
 // t % 2 == g and every head, with its own O^T accumulator; kSplit == true:
 // both groups take every tile, group g the heads [g HG, (g+1) HG), and they
 // share one O^T accumulator (its columns are disjoint by head).
-template <typename E, int GP, bool kSplit>
+template <typename E, int GP, bool kSplit, int D>
 __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) {
-    using C = KCfg<GP>;
+    using C = KCfg<GP, D>;
     constexpr int NQ = C::NQ;
-    constexpr int D = kKD;
     constexpr int HG = kSplit ? GP / 2 : GP;    // heads of one group
     const int G = p.G;
     const int grp = (x.warp - 2) >> 2;
@@ -291,15 +306,14 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             if (rows < kKT && (!kSplit || grp == 0)) {
                 // keys past the piece end: p is 0 there, and 0 * NaN would poison
                 // O^T, so zero those V rows before the P V product reads them
-                const int stg = static_cast<int>(t % kKStages);
-                unsigned char* vb =
-                    smem + C::kOffKV + stg * C::kStageBytes + C::kAtoms * C::kKVAtom;
+                const int stg = static_cast<int>(t % C::kStages);
+                unsigned char* vb = smem + C::kOffKV + stg * C::kStageBytes + C::kOffVAtoms;
                 // 16-byte unit u: row rows + u / (8 kAtoms), atom (u / 8) % kAtoms, chunk u % 8
-                static_assert(C::kAtoms == 2, "two 64-column atoms per row");
 #pragma unroll 1
-                for (int u = st; u < (kKT - rows) * 16; u += kKGroup)
-                    *reinterpret_cast<uint4*>(vb + ((u >> 3) & 1) * C::kKVAtom +
-                                              swz(rows + (u >> 4), u & 7)) = make_uint4(0, 0, 0, 0);
+                for (int u = st; u < (kKT - rows) * 8 * C::kAtoms; u += kKGroup)
+                    *reinterpret_cast<uint4*>(vb + ((u >> 3) % C::kAtoms) * C::kKVAtom +
+                                              swz(rows + u / (8 * C::kAtoms), u & 7)) =
+                        make_uint4(0, 0, 0, 0);
                 fence_proxy_async_smem();
             }
 
@@ -490,7 +504,8 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int h = h0 + j;
-                if (h < G) {
+                // O^T rows >= D (D = 64) are not part of the result
+                if (h < G && key < D) {
                     float v = has0 ? __uint_as_float(o0[j]) * hs[2 * h] : 0.f;
                     if (has1) v = fmaf(hs[2 * h + 1], __uint_as_float(o1[j]), v);
                     if (whole)
@@ -546,13 +561,13 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
 
 // ------------------------------------------------------------------ kernel
 
-template <typename E, int GP, bool kSplit>
-__global__ void __launch_bounds__(kKThreads, 1)
+template <typename E, int GP, bool kSplit, int D>
+__global__ void __launch_bounds__(kKThreads, KCfg<GP, D>::kCtasPerSm)
     td_gqa_keys_kernel(const GqaParams p, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV) {
-    using C = KCfg<GP>;
+    using C = KCfg<GP, D>;
     constexpr int NQ = C::NQ;
-    constexpr int D = kKD;
+    constexpr int kKStages = C::kStages;
     constexpr bool kBF16 = std::is_same<E, __nv_bfloat16>::value;
     extern __shared__ unsigned char smem_raw[];
     // 1024-byte alignment for the swizzled operand blocks
@@ -638,9 +653,10 @@ __global__ void __launch_bounds__(kKThreads, 1)
                             mbar_arrive_expect_tx(fb, C::kStageBytes);
 #pragma unroll
                             for (int a = 0; a < C::kAtoms; ++a) {
-                                tma_load_2d(base + a * C::kKVAtom, &tmK, 64 * a, y, fb, pol);
-                                tma_load_2d(base + (C::kAtoms + a) * C::kKVAtom, &tmV, 64 * a, y,
-                                            fb, pol);
+                                tma_load_2d(base + C::kOffKAtoms + a * C::kKVAtom, &tmK, 64 * a,
+                                            y, fb, pol);
+                                tma_load_2d(base + C::kOffVAtoms + a * C::kKVAtom, &tmV, 64 * a,
+                                            y, fb, pol);
                             }
                             ++issued;
                         }
@@ -666,7 +682,7 @@ __global__ void __launch_bounds__(kKThreads, 1)
             // S^T: A = K tile (K-major), B = Q (K-major); O^T: A = V^T (V tile,
             // D contiguous: MN-major), B = P^T (K-major)
             constexpr uint32_t idS = instr_desc_f16(kBF16 ? 1 : 0, kKT, NQ, 0, 0);
-            constexpr uint32_t idO = instr_desc_f16(kBF16 ? 1 : 0, kKD, NQ, 1, 0);
+            constexpr uint32_t idO = instr_desc_f16(kBF16 ? 1 : 0, kKMO, NQ, 1, 0);
             long long t = 0;    // tiles so far (global)
             long long pc = 0;   // pieces so far
             bool aborted = false;
@@ -705,8 +721,8 @@ __global__ void __launch_bounds__(kKThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < D / 16; ++kk) {
                                 const uint32_t off = static_cast<uint32_t>((kk & 3) * 32);
-                                const uint64_t a =
-                                    smem_desc_sw128(kb + (kk >> 2) * C::kKVAtom + off, 16, 1024);
+                                const uint64_t a = smem_desc_sw128(
+                                    kb + C::kOffKAtoms + (kk >> 2) * C::kKVAtom + off, 16, 1024);
                                 const uint64_t b =
                                     smem_desc_sw128(sQ + (kk >> 2) * C::kQAtom + off, 16, 1024);
                                 umma_f16(dS, a, b, idS, kk > 0 ? 1u : 0u);
@@ -720,8 +736,7 @@ __global__ void __launch_bounds__(kKThreads, 1)
                             fence_after();
                             const long long i = tp - t;
                             const int stage = static_cast<int>(tp % kKStages);
-                            const uint32_t vb =
-                                sKV + stage * C::kStageBytes + C::kAtoms * C::kKVAtom;
+                            const uint32_t vb = sKV + stage * C::kStageBytes + C::kOffVAtoms;
                             const uint32_t pb = sP + static_cast<uint32_t>((tp & 1) * C::kPBytes);
                             // one O^T per group (tiles alternate), or one shared
                             const uint32_t dO = tmem + static_cast<uint32_t>(
@@ -729,7 +744,8 @@ __global__ void __launch_bounds__(kKThreads, 1)
 #pragma unroll
                             for (int kk = 0; kk < kKT / 16; ++kk) {
                                 // 16 keys: rows 16 kk.. of the V tile; the two
-                                // 64-column halves of D are kKVAtom apart
+                                // 64-row halves of M are kKVAtom apart (D = 64:
+                                // the second is the K tile, rows never read)
                                 const uint64_t a =
                                     smem_desc_sw128(vb + kk * 2048, C::kKVAtom, 1024);
                                 const uint64_t b = smem_desc_sw128(
@@ -785,7 +801,7 @@ __global__ void __launch_bounds__(kKThreads, 1)
         // --------------------------------------------------------- softmax
         const KCtx kx{smem, s_full, s_empty, p_full, pv_done, &q_ready, &ctl, abort_flag,
                       tmem, T, x0, x1, P, c, warp, lane, tid};
-        keys_softmax<E, GP, kSplit>(p, kx);
+        keys_softmax<E, GP, kSplit, D>(p, kx);
     }
 
     fence_before();
@@ -797,11 +813,11 @@ __global__ void __launch_bounds__(kKThreads, 1)
     }
 }
 
-template <typename E, int GP, bool kSplit>
+template <typename E, int GP, bool kSplit, int D>
 cudaError_t launch_keys_t(int device, const GqaParams& p, const CUtensorMap& mk,
                           const CUtensorMap& mv, cudaStream_t s) {
-    using C = KCfg<GP>;
-    auto kern = td_gqa_keys_kernel<E, GP, kSplit>;
+    using C = KCfg<GP, D>;
+    auto kern = td_gqa_keys_kernel<E, GP, kSplit, D>;
     static std::atomic<unsigned long long> configured{0};
     const unsigned long long bit = device < 64 ? (1ull << device) : 0ull;
     if (!bit || !(configured.load(std::memory_order_acquire) & bit)) {
@@ -814,30 +830,48 @@ cudaError_t launch_keys_t(int device, const GqaParams& p, const CUtensorMap& mk,
     return cudaGetLastError();
 }
 
-template <typename E>
+template <typename E, int D>
 cudaError_t launch_keys_g(int device, const GqaParams& p, const CUtensorMap& mk,
                           const CUtensorMap& mv, cudaStream_t s) {
     // up to 8 heads a thread keeps every head and the groups alternate tiles;
     // beyond, both groups take every tile with half the heads each
-    if (p.G <= 4) return launch_keys_t<E, 4, false>(device, p, mk, mv, s);
-    if (p.G <= 8) return launch_keys_t<E, 8, false>(device, p, mk, mv, s);
-    if (p.G <= 16) return launch_keys_t<E, 16, true>(device, p, mk, mv, s);
-    return launch_keys_t<E, 32, true>(device, p, mk, mv, s);
+    if (p.G <= 4) return launch_keys_t<E, 4, false, D>(device, p, mk, mv, s);
+    if (p.G <= 8) return launch_keys_t<E, 8, false, D>(device, p, mk, mv, s);
+    if (p.G <= 16) return launch_keys_t<E, 16, true, D>(device, p, mk, mv, s);
+    return launch_keys_t<E, 32, true, D>(device, p, mk, mv, s);
+}
+
+template <int D>
+size_t keys_smem(int G) {
+    return G <= 4 ? KCfg<4, D>::kSmem : G <= 8 ? KCfg<8, D>::kSmem
+                                               : G <= 16 ? KCfg<16, D>::kSmem
+                                                         : KCfg<32, D>::kSmem;
 }
 
 }  // namespace
 
-bool gqa_keys_path(int D, int G) { return D == kKD && G >= 1 && G <= 32; }
+bool gqa_keys_path(int D, int G) { return (D == 64 || D == 128) && G >= 1 && G <= 32; }
 
-size_t gqa_keys_smem_bytes(int G) {
-    return G <= 4 ? KCfg<4>::kSmem : G <= 8 ? KCfg<8>::kSmem : G <= 16 ? KCfg<16>::kSmem
-                                                                         : KCfg<32>::kSmem;
+int gqa_keys_ctas_per_sm(int D, int G) {
+    if (D == 64)
+        return G <= 4 ? KCfg<4, 64>::kCtasPerSm : G <= 8 ? KCfg<8, 64>::kCtasPerSm
+               : G <= 16 ? KCfg<16, 64>::kCtasPerSm : KCfg<32, 64>::kCtasPerSm;
+    return 1;
 }
 
-cudaError_t launch_gqa_keys(int device, int dtype, const GqaParams& p, const CUtensorMap& mk,
-                            const CUtensorMap& mv, cudaStream_t s) {
-    if (dtype == kBF16) return launch_keys_g<__nv_bfloat16>(device, p, mk, mv, s);
-    if (dtype == kF16) return launch_keys_g<__half>(device, p, mk, mv, s);
+size_t gqa_keys_smem_bytes(int D, int G) {
+    return D == 64 ? keys_smem<64>(G) : D == 128 ? keys_smem<128>(G) : 0;
+}
+
+cudaError_t launch_gqa_keys(int device, int dtype, int D, const GqaParams& p,
+                            const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t s) {
+    if (D == 128) {
+        if (dtype == kBF16) return launch_keys_g<__nv_bfloat16, 128>(device, p, mk, mv, s);
+        if (dtype == kF16) return launch_keys_g<__half, 128>(device, p, mk, mv, s);
+    } else if (D == 64) {
+        if (dtype == kBF16) return launch_keys_g<__nv_bfloat16, 64>(device, p, mk, mv, s);
+        if (dtype == kF16) return launch_keys_g<__half, 64>(device, p, mk, mv, s);
+    }
     return cudaErrorInvalidValue;
 }
 

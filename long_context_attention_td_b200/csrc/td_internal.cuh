@@ -93,12 +93,14 @@ cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const C
 // Merge the part records of every split sequence (p.fused_merge == 0).
 cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s);
 // Grouped-query kernel with the keys on the MMA M axis (td_gqa_keys.cu): same
-// parameters and part records, for D == 128 and G <= 32; its K and V tensor
-// maps use boxes of {64 columns, 128 rows}.
+// parameters and part records, for D == 64 or 128 and G <= 32; its K and V
+// tensor maps use boxes of {64 columns, 128 rows}.
 bool gqa_keys_path(int D, int G);
-size_t gqa_keys_smem_bytes(int G);
-cudaError_t launch_gqa_keys(int device, int dtype, const GqaParams& p, const CUtensorMap& mk,
-                            const CUtensorMap& mv, cudaStream_t s);
+// CTAs of that kernel that share one SM (its launch bounds)
+int gqa_keys_ctas_per_sm(int D, int G);
+size_t gqa_keys_smem_bytes(int D, int G);
+cudaError_t launch_gqa_keys(int device, int dtype, int D, const GqaParams& p,
+                            const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t s);
 
 // The split-KV kernel over an FP8 E4M3 K/V cache, q of type q_dtype (kBF16, kF16).
 cudaError_t launch_partial_fp8(int device, int q_dtype, int D, const PartialParams& p,

@@ -2,6 +2,7 @@
 host-side logic (validation, split heuristic, workspace sizing) behaves --
 all without a GPU and without launching anything."""
 import ctypes
+import math
 import os
 import re
 
@@ -114,10 +115,15 @@ def test_auto_split_fills_the_gpu_and_respects_part_size(L):
         P = L.td_auto_split(B, H, N, 128, 1, sms)
         assert P % sms == 0 and P >= sms
         assert L.td_auto_split(B, H, N, 128, 1, 2 * sms) == 2 * P
-    # tiny problem: no part below 64 KiB of K+V, never more parts than keys
+    # tiny problem: no part below 64 KiB of K+V, never more parts than keys, and
+    # no more parts per sequence than keep its merge cheap: floor(sqrt(0.62 N elt))
     P = L.td_auto_split(1, 1, 4096, 512, 0, sms)  # fp32 D=512: 4 KiB per key
-    assert P == min(sms * (P // sms or 1), 4096 * 4096 // 65536) or P <= 256
-    assert 1 <= P <= 256
+    assert P == int(math.sqrt(0.62 * 4096 * 4))      # 100, the measured optimum 64..128
+    fill = L.td_auto_split(1, 1, 1 << 22, 512, 0, sms)  # long sequence: every CTA slot
+    assert fill % sms == 0
+    assert L.td_auto_split(4, 2, 4096, 512, 0, sms) == min(8 * 100, fill)
+    # long sequences never reach the cap
+    assert L.td_auto_split(1, 32, 131072, 128, 1, sms) == 3 * sms
     assert L.td_auto_split(1, 1, 3, 64, 2, sms) == 1
     assert L.td_auto_split(1, 1, 5, 64, 2, sms) <= 5
     for bad in ((0, 1, 1, 128, 1, sms), (1, 1, 0, 128, 1, sms), (1, 1, 8, 96, 1, sms),

@@ -63,9 +63,10 @@ def test_gqa_group_sizes(dtype, D, G):
     run_and_check(w, Hkv)
 
 
-@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 129, 1000])
-def test_gqa_lengths_and_alibi(N):
-    w = Workload("gqa_n", torch.bfloat16, 1, 16, 128, N, alibi=True, seed=400 + N)
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("N", [1, 2, 63, 64, 65, 127, 128, 129, 1000])
+def test_gqa_lengths_and_alibi(N, D):
+    w = Workload("gqa_n", torch.bfloat16, 1, 16, D, N, alibi=True, seed=400 + N + D)
     for n_split in (0, 1, 3):
         run_and_check(w, 2, n_split=n_split)
 
@@ -83,10 +84,18 @@ def test_gqa_merge_of_more_than_a_chunk_of_parts():
     run_and_check(w, 2, parts=2 * 1300)
 
 
-def test_gqa_ragged_with_empty_sequences():
-    w = Workload("gqa_r", torch.bfloat16, 5, 16, 128, 900, alibi=True, seed=600)
+@pytest.mark.parametrize("D", [64, 128])
+def test_gqa_ragged_with_empty_sequences(D):
+    w = Workload("gqa_r", torch.bfloat16, 5, 16, D, 900, alibi=True, seed=600 + D)
     run_and_check(w, 4, lens=[0, 1, 900, 333, 0])
     run_and_check(w, 4, parts=7, lens=[0, 1, 900, 333, 0])
+
+
+def test_gqa_d64_bench_shape_sampled():
+    """The grouped-query D = 64 workload at a reduced length (fp16, B16 Hq32
+    Hkv4, G = 8), every query head against the oracle."""
+    w = Workload("gqa_d64", torch.float16, 16, 32, 64, 8192, seed=1244)
+    run_and_check(w, 4)
 
 
 def test_gqa_multi_query_long():
