@@ -42,7 +42,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from long_context_attention_td_b200.workloads import (WORKLOADS, kv_bytes, kv_lengths,  # noqa: E402
-                                                      make_inputs, prefill_flops)
+                                                      make_inputs, prefill_flops, seqlens_for)
 
 METRIC = "decode attention KV GB/s and % of B200 HBM peak (1 GPU); µs per decode step"
 PREFILL_METRIC = "prefill attention TFLOP/s (4 D FLOPs per visible query-key pair; 1 GPU)"
@@ -251,6 +251,51 @@ def hbm_roofline(achieved, peak, peak_kind, kernel, bytes_per_launch, traffic, t
             "algorithmic_bytes_per_launch": int(bytes_per_launch)}
 
 
+def rotation_copies(bytes_step):
+    """Copies of K and V the timed steps rotate over so that a workload whose
+    K+V fit in L2 is read from HBM: enough that the steps between two uses of
+    one copy read more than twice the L2."""
+    if bytes_step >= 2 * L2_BYTES:
+        return 1
+    return min(64, -(-2 * L2_BYTES // max(bytes_step, 1)))
+
+
+def is_shardable(w):
+    """Workloads the sequence-sharded step takes: multi-head decode (uniform,
+    or ragged without a positional bias)."""
+    if w.prefill or w.kv_fp8 or (w.kv_heads and w.kv_heads != w.H):
+        return False
+    return not (w.ragged is not None and w.alibi)
+
+
+def parallelism_name(world, sharded):
+    return ("sequence-sharded x%d" % world) if sharded else ("replicas x%d" % world)
+
+
+def workload_config(args, w, parallelism):
+    """The `config` object both arms print for a workload: its shape and the
+    L2 handling, all host arithmetic (the same on a box without a GPU)."""
+    if w.prefill:
+        return {"workload": args.workload + ("" if not args.n_keys else "@S=%d" % w.N),
+                "B": w.B, "H": w.H, "D": w.D, "S": w.N, "causal": w.causal, "alibi": w.alibi,
+                "flops_per_step": prefill_flops(w),
+                "l2": "no flush: q, k, v, out per step %.2f GB > 126 MB L2"
+                      % ((3 * 2 + 4) * w.B * w.H * w.N * w.D / 1e9),
+                "parallelism": parallelism}
+    n_split = w.n_split if args.n_split is None else args.n_split
+    bytes_step = kv_bytes(w, seqlens_for(w))
+    n_rot = rotation_copies(bytes_step)
+    return {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % w.N),
+            "B": w.B, "H": w.H, "kv_heads": w.kv_heads or w.H, "D": w.D, "N": w.N,
+            "ragged": w.ragged is not None, "alibi": w.alibi,
+            "n_split": n_split if n_split else "auto", "bytes_per_step": int(bytes_step),
+            "l2": ("no flush: K+V per step %.2f GB > 126 MB L2" % (bytes_step / 1e9)
+                   if n_rot == 1 else
+                   "no flush: steps rotate over %d copies of K+V (%.1f MB each, %.0f MB "
+                   "in all > 2 x 126 MB L2)" % (n_rot, bytes_step / 1e6, n_rot * bytes_step / 1e6)),
+            "parallelism": parallelism}
+
+
 # -------------------------------------------------------------- CPU oracle
 
 def oracle_rate_gqa(inp, w, budget_s, min_s=0.0, threads=0):
@@ -449,9 +494,7 @@ def run_ours(args):
     # a step whose K and V fit in L2 would be timed from L2: rotate over enough
     # distinct copies of K and V that the steps between two uses of one copy
     # read more than twice the L2
-    n_rot = 1
-    if bytes_step < 2 * L2_BYTES:
-        n_rot = min(64, -(-2 * L2_BYTES // max(bytes_step, 1)))
+    n_rot = rotation_copies(bytes_step)
     kv_sets = [(k, v)] + [(k.clone(), v.clone()) for _ in range(n_rot - 1)]
     step_no = [0]
 
@@ -595,17 +638,9 @@ def run_ours(args):
             "dtype": "f32", "input_dtype": (DTYPE_NAME[w.dtype] + " q, e4m3 k/v (f16 products)"
                                             if w.kv_fp8 else DTYPE_NAME[w.dtype]),
             "data": "synthetic",
-            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % N),
-                       "B": B, "H": H, "kv_heads": w.kv_heads or H, "D": D, "N": N,
-                       "ragged": w.ragged is not None, "alibi": w.alibi,
-                       "n_split": n_split if n_split else "auto", "parts": parts,
-                       "bytes_per_step": int(bytes_step),
-                       "l2": ("no flush: K+V per step %.2f GB > 126 MB L2" % (bytes_step / 1e9)
-                              if n_rot == 1 else
-                              "no flush: steps rotate over %d copies of K+V (%.1f MB each, %.0f MB "
-                              "in all > 2 x 126 MB L2)" % (n_rot, bytes_step / 1e6,
-                                                          n_rot * bytes_step / 1e6)),
-                       "parallelism": "replicas x%d" % world},
+            "config": workload_config(args, w.with_(seed=WORKLOADS[args.workload].seed),
+                                      parallelism_name(world, False)),
+            "launch": {"parts": parts},
             "gpu_launches": int(launches), "clocks": clocks, "roofline": roofline, "parity": parity,
             "e2e": e2e, "cpu_baseline": cpu,
         }
@@ -693,12 +728,7 @@ def run_prefill(args):
             "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate",
             "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
-            "config": {"workload": args.workload + ("" if not args.n_keys else "@S=%d" % w.N),
-                       "B": w.B, "H": w.H, "D": w.D, "S": w.N, "causal": w.causal,
-                       "alibi": w.alibi, "flops_per_step": flops,
-                       "l2": "no flush: q, k, v, out per step %.2f GB > 126 MB L2"
-                             % ((3 * 2 + 4) * w.B * w.H * w.N * w.D / 1e9),
-                       "parallelism": "replicas x%d" % world},
+            "config": workload_config(args, w, parallelism_name(world, False)),
             "gpu_launches": int(launches), "clocks": clocks,
             "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak,
                          "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -902,13 +932,10 @@ def run_sharded(args):
                                         (ms_per_step * 1e-3), 1),
             "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f32",
             "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic",
-            "config": {"workload": args.workload + ("" if not args.n_keys else "@N=%d" % w.N),
-                       "B": B, "H": H, "D": D, "N": w.N, "ragged": w.ragged is not None,
-                       "alibi": w.alibi, "bytes_per_step": int(bytes_all),
-                       "l2": "no flush: K+V per rank per step %.2f GB > 126 MB L2"
-                             % (shard_bytes / 1e9),
-                       "parallelism": "sequence-sharded x%d" % world,
-                       "collective": "one all_gather of B*H*(D+1) fp32 per rank (NCCL)"},
+            "config": workload_config(args, w, parallelism_name(world, True)),
+            "launch": {"collective": "one all_gather of B*H*(D+1) fp32 per rank (NCCL)",
+                       "rank_bytes_per_step": int(shard_bytes),
+                       "rank_l2": "K+V per rank per step %.2f GB > 126 MB L2" % (shard_bytes / 1e9)},
             "gpu_launches": int(launches), "clocks": clocks,
             "roofline": hbm_roofline(achieved, peak, peak_kind, kernel_name, shard_bytes, None,
                                      "none: per-rank chunk, not captured"),
@@ -928,7 +955,17 @@ def run_reference(args):
     if rank != 0:
         return
     w = WORKLOADS[args.workload]
-    inp = make_inputs(w, "cpu")
+    if args.n_keys:
+        w = w.with_(N=args.n_keys)
+    sharded = world > 1 and not args.replicas and is_shardable(w)
+    config = workload_config(args, w, parallelism_name(world, sharded or args.shard_seq))
+    # the oracle's sample reads the first rows of the first batch entries only
+    # (one per host core at most): generate just those entries on the host
+    cores = os.cpu_count() or 1
+    plain = not (w.prefill or w.kv_fp8 or (w.kv_heads and w.kv_heads != w.H))
+    b_need = min(w.B, max(1, -(-cores // w.H))) if plain else 1
+    inp = make_inputs(w.with_(B=b_need), "cpu")
+    w = w.with_(B=b_need)
     # each step is a bounded sample so the whole run stays within ~2 minutes
     per_step_budget = max(0.002, 120.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
@@ -948,7 +985,7 @@ def run_reference(args):
         "ms_per_step": round(1e3 * dt / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "input_dtype": DTYPE_NAME[w.dtype], "data": "synthetic", "impl": "reference",
-        "config": {"workload": args.workload, "B": w.B, "H": w.H, "D": w.D, "N": w.N},
+        "config": config,
         "cpu_baseline": {"value": round(value, 6), "unit": unit, "cores": used,
                          "kind": "oracle", "sample": "per step: " + desc},
         "e2e": {"value": round(value, 6), "unit": unit, "h2d_bytes_per_step": 0,
@@ -982,10 +1019,9 @@ def main(argv=None):
         raise SystemExit("--warmup must be >= 3")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     w = WORKLOADS[args.workload]
-    shardable = not (w.prefill or w.kv_fp8 or (w.kv_heads and w.kv_heads != w.H))
     if args.impl == "reference":
         run_reference(args)
-    elif args.shard_seq or (world > 1 and shardable and not args.replicas):
+    elif args.shard_seq or (world > 1 and is_shardable(w) and not args.replicas):
         run_sharded(args)
     elif WORKLOADS[args.workload].prefill:
         run_prefill(args)
