@@ -27,7 +27,8 @@
 //
 // 12 warps in three warpgroups: warpgroup 0 -- warp 0 loads Q and K, warp 2
 // loads V (3-D boxes of {64 columns, 128 rows, 1 sequence}; 2 K and 3 V
-// stages), warp 1 owns TMEM and issues the MMAs, warp 3 idles; warpgroup 1 is
+// stages), warp 1 owns TMEM and issues the MMAs as their inputs become
+// ready, warp 3 idles; warpgroup 1 is
 // the softmax of query tile 0, warpgroup 2 that of query tile 1 (warp w reads
 // TMEM lanes 32 (w % 4) .. + 31).
 #include <cuda.h>
@@ -53,8 +54,8 @@ constexpr int kPThreads = 384;       // 12 warps (two softmax warpgroups)
 // to kRegLow, the softmax warpgroups rise to kRegHigh; 4*32*kRegLow +
 // 8*32*kRegHigh must not exceed the 384 x 168 registers the block is launched
 // with, or the increase would wait for ever
-constexpr int kRegLow = 56;
-constexpr int kRegHigh = 224;
+constexpr int kRegLow = 64;
+constexpr int kRegHigh = 216;
 static_assert(4 * 32 * kRegLow + 8 * 32 * kRegHigh <= kPThreads * 168, "register split");
 constexpr int kKStages = 2;          // K ring depth
 constexpr int kVStages = 3;          // V ring depth (its stage is held until P V is done)
@@ -69,7 +70,8 @@ struct PCfg {
     static constexpr int kOffQ = 0;                       // Q_0, Q_1
     static constexpr int kOffK = 2 * kTileBytes;
     static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-    static constexpr size_t kSmem = size_t(kOffV) + kVStages * kTileBytes + 1024;  // +align
+    static constexpr int kOffRamp = kOffV + kVStages * kTileBytes;  // ALiBi slope * c, 128 floats
+    static constexpr size_t kSmem = size_t(kOffRamp) + kPK * 4 + 1024;  // +align
     static_assert(D == 64 || D == 128, "D");
     static_assert(kSmem <= 232448 - 256, "shared memory");
 };
@@ -97,10 +99,46 @@ __device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem
         : "memory");
 }
 
+// mbarrier phase test that may suspend the thread for up to `ns` nanoseconds
+// while the phase is incomplete (frees the issue slots a polling thread takes)
+__device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 struct PCtl {
     int abort;
     uint32_t tmem;
 };
+
+// ---------------------------------------------- packed fp32 pairs (f32x2)
+
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 
 template <typename E, int D>
 __global__ void __launch_bounds__(kPThreads, 1)
@@ -167,6 +205,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      ::"r"(smem_addr(&ctl.tmem)), "r"(kPTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (p.slopes && tid >= 128 && tid < 128 + kPK) {
+        // the ALiBi ramp slope_h c (log2 units) of key c of a tile; the tile's
+        // offset slope_h (j0 - S + 1) is added to the row's running max instead
+        reinterpret_cast<float*>(smem + C::kOffRamp)[tid - 128] =
+            __ldg(p.slopes + (bh % p.H)) * kLog2e * static_cast<float>(tid - 128);
     }
     fence_before();
     __syncthreads();
@@ -242,17 +286,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
             constexpr uint32_t idS = instr_desc_f16(kBF16 ? 1 : 0, kPQ, kPK, 0, 0);
             constexpr uint32_t idO = instr_desc_f16(kBF16 ? 1 : 0, kPQ, D, 0, 1);
             bool aborted = false;
-            auto wait = [&](uint64_t* bar, uint32_t par) {
-                if (!aborted && !mbar_wait_bounded(smem_addr(bar), par, abort_flag, p.err,
-                                                   TD_DEVERR_WAIT_TIMEOUT))
-                    aborted = true;
-                return !aborted;
-            };
             // S_g of key tile t into TMEM columns [128 g, 128 g + 128)
-            auto issue_s = [&](int g, long long t) {
+            auto issue_s = [&](int g, int t) {
                 const int stage = static_cast<int>(t % kKStages);
-                if (!wait(&k_full[stage], static_cast<uint32_t>((t / kKStages) & 1))) return;
-                fence_after();
                 const uint32_t kb = sK + stage * C::kTileBytes;
                 const uint32_t qb = sQ + g * C::kTileBytes;
                 const uint32_t dS = tmem + static_cast<uint32_t>(g * kPK);
@@ -264,16 +300,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     umma_f16(dS, a, b, idS, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(smem_addr(&s_full[g]));
-                // query tile 1 reads every key tile tile 0 reads and is issued
-                // second, so it releases the K stage unless it has no such tile
-                if (g == 1 || t >= n1) umma_commit(smem_addr(&k_empty[stage]));
             };
             // O_g += P_g V of key tile t, P_g from TMEM columns [128 g, 128 g + 64)
-            auto issue_pv = [&](int g, long long t) {
-                if (!wait(&p_full[g], static_cast<uint32_t>(t & 1))) return;
+            auto issue_pv = [&](int g, int t) {
                 const int stage = static_cast<int>(t % kVStages);
-                if (!wait(&v_full[stage], static_cast<uint32_t>((t / kVStages) & 1))) return;
-                fence_after();
                 const uint32_t vb = sV + stage * C::kTileBytes;
                 const uint32_t pa = tmem + static_cast<uint32_t>(g * kPK);
                 const uint32_t dO = tmem + static_cast<uint32_t>(2 * kPK + g * D);
@@ -284,21 +314,93 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     umma_f16_tmem_a(dO, pa + static_cast<uint32_t>(kk * 8), b, idO,
                                     (t > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (g == 1 || t >= n1) umma_commit(smem_addr(&v_empty[stage]));
-                if (t == (g == 0 ? n0 : n1) - 1) umma_commit(smem_addr(&o_done[g]));
+                if (t == static_cast<int>(g == 0 ? n0 : n1) - 1) umma_commit(smem_addr(&o_done[g]));
             };
-            if (wait(&q_full, 0)) {
+            // Event loop: each group's products go out as soon as their inputs
+            // are ready, so neither softmax group waits behind the other's.
+            // S_g(t) follows P_g V(t - 1) (it overwrites P_g); P_g V(t) needs
+            // P_g(t) written and V(t) landed.  A K (V) stage is released after
+            // its last user: (t < n0) + (t < n1) products read tile t.
+            if (mbar_wait_bounded(smem_addr(&q_full), 0, abort_flag, p.err,
+                                  TD_DEVERR_WAIT_TIMEOUT)) {
                 fence_after();
-                if (n0 > 0) issue_s(0, 0);
-                if (n1 > 0) issue_s(1, 0);
-                for (long long t = 0; t < nt && !aborted; ++t) {
-                    if (t < n0) {
-                        issue_pv(0, t);
-                        if (t + 1 < n0) issue_s(0, t + 1);
+                // tile counters fit 32 bits (S < 2^31 keys)
+                const int ngr[2] = {static_cast<int>(n0), static_cast<int>(n1)};
+                int ts[2] = {0, 0}, tp[2] = {0, 0};
+                // products issued so far on each stage's current tile, 2 bits a stage
+                uint32_t kuse = 0, vuse = 0;
+                static_assert(kKStages <= 16 && kVStages <= 16, "stage use counters");
+                uint64_t t_stall = 0;
+                uint32_t spins = 0;
+                while (!aborted && (tp[0] < ngr[0] || tp[1] < ngr[1])) {
+                    bool progressed = false;
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        if (tp[g] < ts[g]) {
+                            const int t = tp[g];
+                            const int vst = static_cast<int>(t % kVStages);
+                            if (mbar_test(smem_addr(&p_full[g]), static_cast<uint32_t>(t & 1)) &&
+                                mbar_test(smem_addr(&v_full[vst]),
+                                          static_cast<uint32_t>((t / kVStages) & 1))) {
+                                fence_after();
+                                issue_pv(g, t);
+                                const uint32_t sh = 2u * static_cast<uint32_t>(vst);
+                                const uint32_t u = ((vuse >> sh) & 3u) + 1u;
+                                if (u == static_cast<uint32_t>((t < ngr[0]) + (t < ngr[1]))) {
+                                    vuse &= ~(3u << sh);
+                                    umma_commit(smem_addr(&v_empty[vst]));
+                                } else {
+                                    vuse = (vuse & ~(3u << sh)) | (u << sh);
+                                }
+                                ++tp[g];
+                                progressed = true;
+                            }
+                        }
+                        if (ts[g] < ngr[g] && ts[g] == tp[g]) {
+                            const int t = ts[g];
+                            const int kst = static_cast<int>(t % kKStages);
+                            if (mbar_test(smem_addr(&k_full[kst]),
+                                          static_cast<uint32_t>((t / kKStages) & 1))) {
+                                fence_after();
+                                issue_s(g, t);
+                                const uint32_t sh = 2u * static_cast<uint32_t>(kst);
+                                const uint32_t u = ((kuse >> sh) & 3u) + 1u;
+                                if (u == static_cast<uint32_t>((t < ngr[0]) + (t < ngr[1]))) {
+                                    kuse &= ~(3u << sh);
+                                    umma_commit(smem_addr(&k_empty[kst]));
+                                } else {
+                                    kuse = (kuse & ~(3u << sh)) | (u << sh);
+                                }
+                                ++ts[g];
+                                progressed = true;
+                            }
+                        }
                     }
-                    if (t < n1) {
-                        issue_pv(1, t);
-                        if (t + 1 < n1) issue_s(1, t + 1);
+                    if (progressed) {
+                        spins = 0;
+                        t_stall = 0;
+                        continue;
+                    }
+                    // nothing ready: suspend briefly on the P of the group whose
+                    // product is oldest (or on the next K tile), then check the
+                    // time limit and the abort flag
+                    const bool w0 = tp[0] < ts[0], w1 = tp[1] < ts[1];
+                    if (w0 || w1) {
+                        const bool first0 = w0 && (!w1 || tp[0] <= tp[1]);
+                        const int tw = first0 ? tp[0] : tp[1];
+                        mbar_try_wait_ns(smem_addr(first0 ? &p_full[0] : &p_full[1]),
+                                         static_cast<uint32_t>(tw & 1), 100);
+                    }
+                    if ((++spins & 31u) == 0u) {
+                        const uint64_t now = global_timer_ns();
+                        if (t_stall == 0) t_stall = now;
+                        if (*abort_flag) {
+                            aborted = true;
+                        } else if (now - t_stall > kWaitLimitNs) {
+                            atomicOr(p.err, TD_DEVERR_WAIT_TIMEOUT);
+                            *abort_flag = 1;
+                            aborted = true;
+                        }
                     }
                 }
             }
@@ -344,11 +446,16 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // sequence end are -inf (every row sees key j0, so its max is
             // finite).  A tile with every key visible and no bias takes the
             // row max on the raw products (qscale2 > 0 keeps the order) and
-            // forms x_c - m with one fma in the exponential loop; the others
-            // build x_c first.  Maxima run as 8 independent chains.
+            // forms x_c - m with one fma in the exponential loop.  With a bias
+            // the scores are built as x'_c = raw_c qscale2 + slope2 c (the
+            // ramp in shared memory) and the tile's offset ofs = slope2 (j0 -
+            // S + 1) joins the max: x_c - m = x'_c - (m - ofs).  Maxima run as
+            // 8 independent chains.
             const long long j0 = t * kPK;
             const int cmax = static_cast<int>(jmax - j0 < kPK - 1 ? jmax - j0 : kPK - 1);
             const bool plain = p.slopes == nullptr && __all_sync(0xffffffffu, cmax == kPK - 1);
+            const bool masked = __any_sync(0xffffffffu, cmax < kPK - 1);
+            const float ofs = slope2 * static_cast<float>(j0 - p.S + 1);
             float mx8[8];
             if (plain) {
 #pragma unroll
@@ -356,28 +463,40 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
                 for (int c = 8; c < kPK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
             } else {
-                const float base = slope2 * static_cast<float>(j0 - p.S + 1);
+                const float* ramp = reinterpret_cast<const float*>(smem + C::kOffRamp);
 #pragma unroll
                 for (int c = 0; c < 8; ++c) mx8[c] = kNegInf;
                 auto build = [&](auto masked_c) {
                     constexpr bool kMasked = decltype(masked_c)::value;
 #pragma unroll
-                    for (int c = 0; c < kPK; ++c) {
-                        float x = fmaf(__uint_as_float(sr[c]), qscale2,
-                                       fmaf(slope2, static_cast<float>(c), base));
-                        if (kMasked) x = c <= cmax ? x : kNegInf;
-                        sr[c] = __float_as_uint(x);
-                        mx8[c & 7] = fmaxf(mx8[c & 7], x);
+                    for (int c4 = 0; c4 < kPK; c4 += 4) {
+                        const float4 b4 = p.slopes ? *reinterpret_cast<const float4*>(ramp + c4)
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                        float x[4];
+                        const uint64_t sc2 = pk2(qscale2, qscale2);
+                        upk2(fma2(pk2(__uint_as_float(sr[c4]), __uint_as_float(sr[c4 + 1])), sc2,
+                                  pk2(b4.x, b4.y)),
+                             x[0], x[1]);
+                        upk2(fma2(pk2(__uint_as_float(sr[c4 + 2]), __uint_as_float(sr[c4 + 3])),
+                                  sc2, pk2(b4.z, b4.w)),
+                             x[2], x[3]);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int c = c4 + u;
+                            if (kMasked) x[u] = c <= cmax ? x[u] : kNegInf;
+                            sr[c] = __float_as_uint(x[u]);
+                            mx8[c & 7] = fmaxf(mx8[c & 7], x[u]);
+                        }
                     }
                 };
-                if (__any_sync(0xffffffffu, cmax < kPK - 1))
+                if (masked)
                     build(std::true_type{});
                 else
                     build(std::false_type{});
             }
             float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
                              fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-            if (plain) mt *= qscale2;
+            mt = plain ? mt * qscale2 : mt + ofs;
             // move this row's max when the tile exceeds it by more than the
             // threshold (always on the first tile)
             const bool need = mt > thr;
@@ -402,21 +521,27 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 thr = mt + kPRescale;
             }
             // p rounded to the input type, two keys per 32-bit column, over the
-            // first 64 columns of S_g; the row sum over 4 independent partials
-            float ls[4] = {0.f, 0.f, 0.f, 0.f};
+            // first 64 columns of S_g, and the row sum over independent partials
+            // (masked keys give ex2(-inf) = 0)
+            uint64_t ls2[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
             auto exps = [&](auto plain_c) {
                 constexpr bool kPlain = decltype(plain_c)::value;
+                const float mneg = plain ? -m : -(m - ofs);
+                const uint64_t sc2 = pk2(qscale2, qscale2);
+                const uint64_t nm2 = pk2(mneg, mneg);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t w[32];
 #pragma unroll
                     for (int y = 0; y < 32; ++y) {
-                        // masked keys give ex2(-inf) = 0
                         const float a0 = __uint_as_float(sr[64 * h + 2 * y]);
                         const float a1 = __uint_as_float(sr[64 * h + 2 * y + 1]);
-                        const float e0 = ex2(kPlain ? fmaf(a0, qscale2, -m) : a0 - m);
-                        const float e1 = ex2(kPlain ? fmaf(a1, qscale2, -m) : a1 - m);
-                        ls[y & 3] += e0 + e1;
+                        const uint64_t x = kPlain ? fma2(pk2(a0, a1), sc2, nm2)
+                                                  : add2(pk2(a0, a1), nm2);
+                        float x0, x1;
+                        upk2(x, x0, x1);
+                        const float e0 = ex2(x0), e1 = ex2(x1);
+                        ls2[y & 1] = add2(ls2[y & 1], pk2(e0, e1));
                         if (kBF16)
                             asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w[y]) : "f"(e1), "f"(e0));
                         else
@@ -429,7 +554,12 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 exps(std::true_type{});
             else
                 exps(std::false_type{});
-            lx += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+            {
+                float a0, a1, b0, b1;
+                upk2(ls2[0], a0, a1);
+                upk2(ls2[1], b0, b1);
+                lx += (a0 + a1) + (b0 + b1);
+            }
             tmem_wait_st();
             fence_before();
             __syncwarp();
