@@ -80,3 +80,17 @@ def test_profiled_traffic_needs_the_current_source_hash(tmp_path, monkeypatch):
     assert bench.profiled_traffic("wl", "unknown_kernel") is None
     monkeypatch.setattr(bench, "kernel_source_hash", lambda k: "fedcba9876543210")
     assert bench.profiled_traffic("wl", "td_partial_kernel") is None
+
+
+def test_reference_arm_prints_the_config_of_the_cuda_arm(capsys):
+    """Both arms build `config` with workload_config (host arithmetic only), so
+    the driver can pair their lines; the reference arm's sample stays small."""
+    import argparse
+    import json
+    for wl in ("gist_f32_d512_n4k", "prefill_bf16_alibi_b4_h16_d128_s4k"):
+        bench.main(["--impl", "reference", "--steps", "3", "--warmup", "3", "--workload", wl])
+        line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+        args = argparse.Namespace(workload=wl, n_keys=0, n_split=None)
+        expect = bench.workload_config(args, WORKLOADS[wl], bench.parallelism_name(1, False))
+        assert line["impl"] == "reference" and line["config"] == expect
+        assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["value"] > 0
