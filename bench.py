@@ -55,7 +55,6 @@ DTYPE_NAME = {torch.float32: "f32", torch.bfloat16: "bf16", torch.float16: "f16"
 KERNEL_SOURCES = {
     "td_partial_kernel": ["td_partial.cu", "td_device.cuh", "td_internal.cuh"],
     "td_gqa_keys_kernel": ["td_gqa_keys.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
-    "td_gqa_kernel": ["td_gqa.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
     "td_prefill_kernel": ["td_prefill.cu", "td_tc.cuh", "td_device.cuh", "td_internal.cuh"],
 }
 

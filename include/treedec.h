@@ -391,7 +391,7 @@ TD_API void td_release_workspace(void);
  * reported by the decode call as TD_ERR_CUDA.
  *
  * td_last_kernel -- name of the main kernel this thread's last successful
- * launch used ("td_partial_kernel", "td_gqa_keys_kernel", "td_gqa_kernel",
+ * launch used ("td_partial_kernel", "td_gqa_keys_kernel",
  * "td_tree_combine_kernel", "td_merge_shards_kernel", "td_empty_state_kernel",
  * "td_prefill_kernel", "td_partial_kernel (fp8 kv)";
  * "" before the first).  Static storage.

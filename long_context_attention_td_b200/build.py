@@ -14,7 +14,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libtreedec.so")
-SOURCES = ["td_partial.cu", "td_combine.cu", "td_gqa.cu", "td_gqa_keys.cu", "td_prefill.cu",
+SOURCES = ["td_partial.cu", "td_combine.cu", "td_gqa_combine.cu", "td_gqa_keys.cu", "td_prefill.cu",
            "td_api.cu", "td_static.cu"]
 HEADERS = ["td_internal.cuh", "td_device.cuh", "td_tc.cuh"]
 

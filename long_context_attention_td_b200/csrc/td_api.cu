@@ -346,13 +346,10 @@ td_status decode_impl(const Req& r) {
 
 // ------------------------------------------------------------- grouped-query
 
-constexpr int kGqaCtasPerSm = 1;
-// parts-per-sequence x group size above which the merge runs as its own kernel
-// (the last CTA of a sequence merges its query heads one after another; the
-// combine kernel spreads them over the SMs, worth its launch much earlier for
-// the keys-on-M kernel, whose main loop ends sooner)
-constexpr long long kGqaSeparateMerge = 128;
-constexpr long long kGqaKeysSeparateMerge = 16;
+// parts-per-sequence x group size from which the merge runs as its own kernel
+// (the last CTA of a sequence would merge its query heads one after another; the
+// combine kernel spreads them over the SMs)
+constexpr long long kGqaSeparateMerge = 16;
 
 // [error word][tickets][segment descriptors: 3 int32 each][part records]
 size_t gqa_desc_region(long long BHkv) { return align_up(static_cast<size_t>(BHkv) * 12, 256); }
@@ -363,10 +360,20 @@ size_t gqa_ws_bytes_for(long long BHkv, int G, int D, long long parts) {
                static_cast<size_t>(D + 3) * sizeof(float);
 }
 
+// Head chunks of a group on the grouped-query kernel and the heads per chunk.
+void gqa_chunking(int G, int* chunks, int* gc) {
+    *chunks = td::gqa_keys_chunks(G);
+    *gc = (G + *chunks - 1) / *chunks;
+}
+
 long long gqa_auto_parts(long long T, int D, int G, int num_sms) {
     if (T <= 0) return 1;
-    const int per_sm = td::gqa_keys_path(D, G) ? td::gqa_keys_ctas_per_sm(D, G) : kGqaCtasPerSm;
-    const long long fill = static_cast<long long>(num_sms) * per_sm;
+    int chunks = 1, gc = G;
+    gqa_chunking(G, &chunks, &gc);
+    const int per_sm = td::gqa_keys_ctas_per_sm(D, gc);
+    // each part runs as `chunks` CTAs: fill the SMs with parts x chunks CTAs
+    long long fill = static_cast<long long>(num_sms) * per_sm / chunks;
+    if (fill < 1) fill = 1;
     const long long bytes_per_key = 2LL * D * 2;
     long long by_size = T / (td::kMinPartBytes / bytes_per_key);
     if (by_size < 1) by_size = 1;
@@ -483,10 +490,9 @@ td_status gqa_impl(const GqaReq& r) {
     if (!mul_fits(P + 1, BHkv * r.N)) return TD_ERR_INVALID_ARG;
     const int G = r.Hq / r.Hkv;
     const size_t need = gqa_ws_bytes_for(BHkv, G, r.D, P);
-    // keys on the MMA M axis (128-key tiles) where that kernel applies, else
-    // query heads on M (64-key tiles)
-    const bool keys_path = td::gqa_keys_path(r.D, G);
-    const int box_rows = keys_path ? 128 : 64;
+    // the keys go on the MMA M axis in tiles of 128: boxes of 128 rows
+    if (!td::gqa_keys_path(r.D, G)) return TD_ERR_UNSUPPORTED;
+    const int box_rows = 128;
     CUtensorMap mk, mv;
     st = make_kv_map(&mk, r.k, BHkv * r.N, r.D, r.dtype, box_rows);
     if (st != TD_OK) return st;
@@ -518,15 +524,12 @@ td_status gqa_impl(const GqaReq& r) {
     // job; when many CTAs share a sequence and many query heads share it, a
     // second kernel spreads the merge over one CTA per (sequence, query head).
     const long long per_seg = (P + BHkv - 1) / BHkv + 1;  // parts touching a sequence
-    p.fused_merge = per_seg * G < (keys_path ? kGqaKeysSeparateMerge : kGqaSeparateMerge) ? 1 : 0;
-    st = cuda_status(launch_main(r.stream, keys_path ? "td_gqa_keys_kernel" : "td_gqa_kernel",
-                                 [&] {
-                                     return keys_path
-                                                ? td::launch_gqa_keys(dev, r.dtype, r.D, p, mk,
-                                                                      mv, r.stream)
-                                                : td::launch_gqa(dev, r.dtype, r.D, p, mk, mv,
-                                                                 r.stream);
-                                 }));
+    p.fused_merge = per_seg * G < kGqaSeparateMerge ? 1 : 0;
+    gqa_chunking(G, &p.chunks, &p.gc);
+    if (!mul_fits(P, p.chunks) || P * p.chunks > 0x7fffffffLL) return TD_ERR_INVALID_ARG;
+    st = cuda_status(launch_main(r.stream, "td_gqa_keys_kernel", [&] {
+        return td::launch_gqa_keys(dev, r.dtype, r.D, p, mk, mv, r.stream);
+    }));
     if (st != TD_OK || p.fused_merge) return st;
     return cuda_status(launch_aux([&] { return td::launch_gqa_combine(r.D, p, r.stream); }));
 }

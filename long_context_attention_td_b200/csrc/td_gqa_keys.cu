@@ -33,7 +33,11 @@
 //               MMAs from one lane, signalling completion with tcgen05.commit;
 //   warps 2-5   softmax group 0 (even tiles), warps 6-9 group 1 (odd tiles);
 //               warp w reads TMEM lanes 32 (w % 4) .. + 31.
-// Used for D = 64 or 128 and G <= 32; td_gqa covers the other shapes.
+// Used for every grouped-query shape (D = 64 or 128, G <= 128): a group of
+// more than 32 heads is cut into chunks of at most 32 heads, one CTA per
+// (part, chunk) over the part's keys; the chunks of a part have adjacent block
+// indices, so they run at the same time and the later ones read the K/V tiles
+// from L2.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -190,6 +194,7 @@ __device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, 
 }
 
 struct KCtx {
+    int g_eff, h_off;        // heads of this CTA's chunk and the first of them
     unsigned char* smem;
     uint64_t* s_full;
     uint64_t* s_empty;
@@ -214,7 +219,9 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
     using C = KCfg<GP, D>;
     constexpr int NQ = C::NQ;
     constexpr int HG = kSplit ? GP / 2 : GP;    // heads of one group
-    const int G = p.G;
+    const int G = x.g_eff;                      // heads of this CTA (its chunk)
+    const int Gall = p.G;                       // heads of the kv head's group
+    const int h_off = x.h_off;                  // first head of the chunk
     const int grp = (x.warp - 2) >> 2;
     const int hb = kSplit ? grp * HG : 0;       // first head of this group
     const int quarter = x.warp & 3;             // TMEM lane quarter of this warp
@@ -250,7 +257,8 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         const long long nt = (j1 - j0 + kKT - 1) / kKT;
         const bool whole = (j0 == 0 && j1 == w.len);
         const long long qrow0 = static_cast<long long>(w.b) * p.Hq +
-                                static_cast<long long>(w.h) * G;   // first query row
+                                static_cast<long long>(w.h) * Gall;  // group's first query row
+        const long long qrow = qrow0 + h_off;                         // this chunk's first
         float* stats = stats_all + (pc & 1) * (2 * 4 * GP * 2 + 2 * GP);
         float* st_l = stats;                      // [grp][head]
         float* st_m = stats + 2 * 4 * GP * 2;     // [grp][head]
@@ -258,7 +266,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         // Q rows of this kv head's group, K-major SW128 (rows >= G stay zero)
         if (grp == 0) {
             const uint4* qg = reinterpret_cast<const uint4*>(static_cast<const E*>(p.q) +
-                                                             qrow0 * D);
+                                                             qrow * D);
             for (int u = st; u < G * (D / 8); u += kKGroup) {
                 const int g = u / (D / 8);
                 const int cc = u - g * (D / 8);
@@ -274,7 +282,9 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         float* slope2 = reinterpret_cast<float*>(smem + C::kOffSlopes) + grp * GP;
         if (p.slopes) {
             if (st < HG)
-                slope2[st] = hb + st < G ? __ldg(p.slopes + w.h * G + hb + st) * kLog2e : 0.f;
+                slope2[st] = hb + st < G
+                                 ? __ldg(p.slopes + w.h * Gall + h_off + hb + st) * kLog2e
+                                 : 0.f;
             named_bar_sync(bar_grp, kKGroup);
         }
         // per head: running max m (uniform in the group; moved when a score
@@ -467,7 +477,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         const bool has0 = kSplit || nt >= 2 || (t_first & 1) == 0;
         const bool has1 = !kSplit && (nt >= 2 || (t_first & 1) == 1);
         const int slot = pc == 0 ? 0 : 1;  // the CTA's first piece uses slot 0
-        float* const part0 = p.part + (x.c * 2 + slot) * G * (D + 3);
+        float* const part0 = p.part + ((x.c * 2 + slot) * Gall + h_off) * (D + 3);
         // per head, once: the merged max M and sum L of both groups, and the
         // weights of the two O^T accumulators in the output (split mode: one
         // accumulator, already relative to the owning group's max)
@@ -482,7 +492,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             if (whole) {
                 a0 /= L;
                 a1 /= L;
-                if (p.lse) p.lse[qrow0 + h] = (M + log2f(L)) * kLn2;
+                if (p.lse) p.lse[qrow + h] = (M + log2f(L)) * kLn2;
             } else {
                 float* rec = part0 + h * (D + 3);
                 rec[D] = M;
@@ -509,7 +519,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                     float v = has0 ? __uint_as_float(o0[j]) * hs[2 * h] : 0.f;
                     if (has1) v = fmaf(hs[2 * h + 1], __uint_as_float(o1[j]), v);
                     if (whole)
-                        p.out[(qrow0 + h) * D + key] = v;
+                        p.out[(qrow + h) * D + key] = v;
                     else
                         part0[h * (D + 3) + key] = v;
                 }
@@ -519,7 +529,7 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
         if (!p.fused_merge) {
             // the CTA holding the sequence's first key describes its parts for
             // the combine kernel (one part: already written, nothing to merge)
-            if (grp == 0 && j0 == 0 && st == 0) {
+            if (grp == 0 && j0 == 0 && st == 0 && h_off == 0) {
                 const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
                 const long long c_lo = gpart_of(w.start, x.T, x.P);
                 const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
@@ -534,7 +544,8 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
             if (grp == 0) {
                 const long long c_lo = gpart_of(w.start, x.T, x.P);
                 const long long c_hi = gpart_of(w.start + w.len - 1, x.T, x.P);
-                const int n = static_cast<int>(c_hi - c_lo + 1);
+                // every chunk CTA of every part of the sequence takes a ticket
+                const int n = static_cast<int>(c_hi - c_lo + 1) * p.chunks;
                 const long long seg = static_cast<long long>(w.b) * p.Hkv + w.h;
                 if (st == 0) {
                     const int prev = atomicAdd(p.tickets + seg, 1);
@@ -546,9 +557,10 @@ __device__ __forceinline__ void keys_softmax(const GqaParams& p, const KCtx& x) 
                 if (x.ctl->last) {
                     __threadfence();
                     const int first_slot = gpart_start(c_lo, x.T, x.P) < w.start ? 1 : 0;
-                    for (int gg = 0; gg < G; ++gg) {
-                        const GSlotAcc acc{p.part, c_lo, first_slot, G, gg, D};
-                        tree_merge(acc, n, D, st, kKGroup, scratch, kKScratch, kBarG0,
+                    const int nparts = n / p.chunks;
+                    for (int gg = 0; gg < Gall; ++gg) {
+                        const GSlotAcc acc{p.part, c_lo, first_slot, Gall, gg, D};
+                        tree_merge(acc, nparts, D, st, kKGroup, scratch, kKScratch, kBarG0,
                                    p.out + (qrow0 + gg) * D, p.lse ? p.lse + qrow0 + gg : nullptr);
                     }
                 }
@@ -579,7 +591,11 @@ __global__ void __launch_bounds__(kKThreads, KCfg<GP, D>::kCtasPerSm)
     __shared__ GCtl ctl;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const long long c = blockIdx.x;
+    // part c and head chunk of this CTA (chunks of a part are adjacent)
+    const long long c = blockIdx.x / p.chunks;
+    const int chunk = static_cast<int>(blockIdx.x % p.chunks);
+    const int h_off = chunk * p.gc;
+    const int g_eff = p.G - h_off < p.gc ? p.G - h_off : p.gc;
     const long long P = p.P;
 
     if (tid == 0) {
@@ -799,8 +815,8 @@ __global__ void __launch_bounds__(kKThreads, KCfg<GP, D>::kCtasPerSm)
         __syncwarp();
     } else {
         // --------------------------------------------------------- softmax
-        const KCtx kx{smem, s_full, s_empty, p_full, pv_done, &q_ready, &ctl, abort_flag,
-                      tmem, T, x0, x1, P, c, warp, lane, tid};
+        const KCtx kx{g_eff, h_off, smem, s_full, s_empty, p_full, pv_done, &q_ready, &ctl,
+                      abort_flag, tmem, T, x0, x1, P, c, warp, lane, tid};
         keys_softmax<E, GP, kSplit, D>(p, kx);
     }
 
@@ -826,7 +842,7 @@ cudaError_t launch_keys_t(int device, const GqaParams& p, const CUtensorMap& mk,
         if (e != cudaSuccess) return e;
         configured.fetch_or(bit, std::memory_order_acq_rel);
     }
-    kern<<<static_cast<unsigned>(p.P), kKThreads, C::kSmem, s>>>(p, mk, mv);
+    kern<<<static_cast<unsigned>(p.P * p.chunks), kKThreads, C::kSmem, s>>>(p, mk, mv);
     return cudaGetLastError();
 }
 
@@ -835,9 +851,9 @@ cudaError_t launch_keys_g(int device, const GqaParams& p, const CUtensorMap& mk,
                           const CUtensorMap& mv, cudaStream_t s) {
     // up to 8 heads a thread keeps every head and the groups alternate tiles;
     // beyond, both groups take every tile with half the heads each
-    if (p.G <= 4) return launch_keys_t<E, 4, false, D>(device, p, mk, mv, s);
-    if (p.G <= 8) return launch_keys_t<E, 8, false, D>(device, p, mk, mv, s);
-    if (p.G <= 16) return launch_keys_t<E, 16, true, D>(device, p, mk, mv, s);
+    if (p.gc <= 4) return launch_keys_t<E, 4, false, D>(device, p, mk, mv, s);
+    if (p.gc <= 8) return launch_keys_t<E, 8, false, D>(device, p, mk, mv, s);
+    if (p.gc <= 16) return launch_keys_t<E, 16, true, D>(device, p, mk, mv, s);
     return launch_keys_t<E, 32, true, D>(device, p, mk, mv, s);
 }
 
@@ -850,12 +866,14 @@ size_t keys_smem(int G) {
 
 }  // namespace
 
-bool gqa_keys_path(int D, int G) { return (D == 64 || D == 128) && G >= 1 && G <= 32; }
+bool gqa_keys_path(int D, int G) { return (D == 64 || D == 128) && G >= 1 && G <= 128; }
 
-int gqa_keys_ctas_per_sm(int D, int G) {
+int gqa_keys_chunks(int G) { return (G + 31) / 32; }
+
+int gqa_keys_ctas_per_sm(int D, int gc) {
     if (D == 64)
-        return G <= 4 ? KCfg<4, 64>::kCtasPerSm : G <= 8 ? KCfg<8, 64>::kCtasPerSm
-               : G <= 16 ? KCfg<16, 64>::kCtasPerSm : KCfg<32, 64>::kCtasPerSm;
+        return gc <= 4 ? KCfg<4, 64>::kCtasPerSm : gc <= 8 ? KCfg<8, 64>::kCtasPerSm
+               : gc <= 16 ? KCfg<16, 64>::kCtasPerSm : KCfg<32, 64>::kCtasPerSm;
     return 1;
 }
 

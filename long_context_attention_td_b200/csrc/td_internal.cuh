@@ -68,7 +68,8 @@ struct PartialParams {
                                  // (tests the bounded-wait failure path); -1: off
 };
 
-// Grouped-query kernel (td_gqa.cu): Hq = G * Hkv query heads over Hkv kv heads.
+// Grouped-query decode (td_gqa_keys.cu, merge in td_gqa_combine.cu): Hq = G * Hkv
+// query heads over Hkv kv heads.
 struct GqaParams {
     const void* q;           // [B, Hq, 1, D]
     float* out;              // [B, Hq, 1, D]
@@ -85,19 +86,21 @@ struct GqaParams {
     int* seg_desc;           // [B * Hkv][3]: first part, parts, slot of the first part
     int fused_merge;         // 1: last CTA merges (ticket); 0: td_gqa_combine merges
     int* err;
+    int chunks;              // keys-on-M kernel: the group's heads in this many chunks,
+    int gc;                  // of gc heads (the last may be shorter), one CTA per (part,
+                             // chunk); 1 and G otherwise
 };
-size_t gqa_smem_bytes(int D);
-// K and V tensor maps: 2-D [B*Hkv*N rows, D columns], box {64, 64}, 128-byte swizzle.
-cudaError_t launch_gqa(int device, int dtype, int D, const GqaParams& p, const CUtensorMap& mk,
-                       const CUtensorMap& mv, cudaStream_t s);
 // Merge the part records of every split sequence (p.fused_merge == 0).
 cudaError_t launch_gqa_combine(int D, const GqaParams& p, cudaStream_t s);
-// Grouped-query kernel with the keys on the MMA M axis (td_gqa_keys.cu): same
-// parameters and part records, for D == 64 or 128 and G <= 32; its K and V
-// tensor maps use boxes of {64 columns, 128 rows}.
+// The grouped-query kernel, keys on the MMA M axis (td_gqa_keys.cu), for D == 64
+// or 128 and G <= 128 (groups of more than 32 heads in chunks of at most 32,
+// one CTA per part and chunk); its K and V tensor maps are 2-D [B*Hkv*N rows,
+// D columns] with boxes of {64 columns, 128 rows} and 128-byte swizzle.
 bool gqa_keys_path(int D, int G);
-// CTAs of that kernel that share one SM (its launch bounds)
-int gqa_keys_ctas_per_sm(int D, int G);
+// head chunks of a group of G and heads per chunk on that kernel
+int gqa_keys_chunks(int G);
+// CTAs of that kernel that share one SM (its launch bounds) for chunks of gc heads
+int gqa_keys_ctas_per_sm(int D, int gc);
 size_t gqa_keys_smem_bytes(int D, int G);
 cudaError_t launch_gqa_keys(int device, int dtype, int D, const GqaParams& p,
                             const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t s);

@@ -87,7 +87,10 @@ WORKLOADS = {
     # grouped-query decode with D = 64: 32 query heads over 4 kv heads, 16 sequences of 64K keys
     "gqa_f16_b16_h32_kv4_d64_n64k": Workload("gqa_f16_b16_h32_kv4_d64_n64k", torch.float16, 16,
                                              32, 64, 65536, seed=1244, kv_heads=4),
-    # multi-query decode with 64 query heads (more than 32: the heads-on-M kernel)
+    # multi-query decode with 48 query heads per kv head (more than 32 heads in one group)
+    "mqa_bf16_h48_kv1_d128_n256k": Workload("mqa_bf16_h48_kv1_d128_n256k", torch.bfloat16, 1, 48,
+                                            128, 1 << 18, seed=1246, kv_heads=1),
+    # multi-query decode with 64 query heads (more than 32 heads in one group)
     "mqa_bf16_h64_kv1_d128_n256k": Workload("mqa_bf16_h64_kv1_d128_n256k", torch.bfloat16, 1, 64,
                                             128, 1 << 18, seed=1245, kv_heads=1),
     # the bench decode shape with an FP8 (E4M3) K/V cache and per-head scales
