@@ -252,7 +252,7 @@ TD_API td_status td_merge_shards(const float *states, int W, int B, int H, int D
  *   q, k, v  device [B,H,S,D] bf16 or fp16 (dtype), row-major, 16-byte aligned;
  *   out      device fp32 [B,H,S,D], 16-byte aligned; lse device fp32 [B,H,S] or NULL;
  *   alibi_slopes device fp32 [H] or NULL.
- *   D in {64, 128}; S >= 1; B*H*ceil(S/128) < 2^31.
+ *   D in {64, 128}; 1 <= S <= 2^31 - 257; B*H*ceil(S/128) < 2^31.
  * Errors: TD_ERR_INVALID_ARG / TD_ERR_UNSUPPORTED before any launch; a bounded
  * wait that ran out sets TD_DEVERR_WAIT_TIMEOUT (td_check_device_error).
  */

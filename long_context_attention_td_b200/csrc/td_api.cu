@@ -567,8 +567,9 @@ td_status prefill_validate(const void* q, const void* k, const void* v, const fl
         (lse && !aligned(lse, 4)) || (slopes && !aligned(slopes, 4)))
         return TD_ERR_INVALID_ARG;
     const long long BH = static_cast<long long>(B) * H;
-    // tensor-map coordinates are 32-bit; the grid is B*H*ceil(S/128) CTAs
-    if (S > 0x7fffffffLL || BH > 0x7fffffffLL || !mul_fits(BH, S) ||
+    // tensor-map coordinates and the kernel's key indices are 32-bit (a tile
+    // index times 128 stays below 2^31); the grid is B*H*ceil(S/128) CTAs
+    if (S > 0x7fffffffLL - 256 || BH > 0x7fffffffLL || !mul_fits(BH, S) ||
         BH * ((S + 127) / 128) > 0x7fffffffLL || !mul_fits(BH * S, static_cast<long long>(D) * 4))
         return TD_ERR_INVALID_ARG;
     return TD_OK;

@@ -113,6 +113,13 @@ __device__ __forceinline__ bool mbar_try_wait_ns(uint32_t bar, uint32_t parity, 
     return ok != 0;
 }
 
+// max of three (one instruction on sm_100)
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 struct PCtl {
     int abort;
     uint32_t tmem;
@@ -206,11 +213,13 @@ __global__ void __launch_bounds__(kPThreads, 1)
                      ::"r"(smem_addr(&ctl.tmem)), "r"(kPTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (p.slopes && tid >= 128 && tid < 128 + kPK) {
-        // the ALiBi ramp slope_h c (log2 units) of key c of a tile; the tile's
-        // offset slope_h (j0 - S + 1) is added to the row's running max instead
+    if (tid >= 128 && tid < 128 + kPK) {
+        // the ALiBi ramp slope_h c (log2 units) of key c of a tile, zero without
+        // a bias; the tile's offset slope_h (j0 - S + 1) is added to the row's
+        // running max instead
         reinterpret_cast<float*>(smem + C::kOffRamp)[tid - 128] =
-            __ldg(p.slopes + (bh % p.H)) * kLog2e * static_cast<float>(tid - 128);
+            p.slopes ? __ldg(p.slopes + (bh % p.H)) * kLog2e * static_cast<float>(tid - 128)
+                     : 0.f;
     }
     fence_before();
     __syncthreads();
@@ -430,7 +439,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
                 aborted = true;
         };
         float m = kNegInf, thr = kNegInf, lx = 0.f;
-        const long long jmax = p.causal ? (i < p.S - 1 ? i : p.S - 1) : p.S - 1;
+        // key indices fit 32 bits (the host keeps S + 256 < 2^31)
+        const int jmax = static_cast<int>(p.causal ? (i < p.S - 1 ? i : p.S - 1) : p.S - 1);
+        const int S1 = static_cast<int>(p.S - 1);
         for (long long t = 0; t < ng; ++t) {
             wait(&s_full[g], static_cast<uint32_t>(t & 1));
             fence_after();
@@ -444,58 +455,58 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // scores in log2 units: x_c = raw_c qscale2 + slope2 (j0 + c - S + 1);
             // keys past the row's last visible key (causal) or past the
             // sequence end are -inf (every row sees key j0, so its max is
-            // finite).  A tile with every key visible and no bias takes the
-            // row max on the raw products (qscale2 > 0 keeps the order) and
-            // forms x_c - m with one fma in the exponential loop.  With a bias
-            // the scores are built as x'_c = raw_c qscale2 + slope2 c (the
-            // ramp in shared memory) and the tile's offset ofs = slope2 (j0 -
-            // S + 1) joins the max: x_c - m = x'_c - (m - ofs).  Maxima run as
-            // 8 independent chains.
-            const long long j0 = t * kPK;
-            const int cmax = static_cast<int>(jmax - j0 < kPK - 1 ? jmax - j0 : kPK - 1);
+            // finite).  One code path serves every tile (a compact loop body
+            // keeps the instruction stream in cache): a tile with every key
+            // visible and no bias keeps the raw products in sr, takes the row
+            // max on them (qscale2 > 0 keeps the order) and forms x_c - m with
+            // one fma in the exponent loop; any other tile first rewrites sr as
+            // x'_c = raw_c qscale2 + slope2 c (the ramp in shared memory, -inf
+            // where masked), and the tile's offset ofs = slope2 (j0 - S + 1)
+            // joins the max: x_c - m = x'_c - (m - ofs).  The max runs as 8
+            // independent chains of three-input maxima.
+            const int j0 = static_cast<int>(t) * kPK;
+            const int cmax = jmax - j0 < kPK - 1 ? jmax - j0 : kPK - 1;
             const bool plain = p.slopes == nullptr && __all_sync(0xffffffffu, cmax == kPK - 1);
-            const bool masked = __any_sync(0xffffffffu, cmax < kPK - 1);
-            const float ofs = slope2 * static_cast<float>(j0 - p.S + 1);
-            float mx8[8];
-            if (plain) {
-#pragma unroll
-                for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
-#pragma unroll
-                for (int c = 8; c < kPK; ++c) mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(sr[c]));
-            } else {
+            const float ofs = slope2 * static_cast<float>(j0 - S1);
+            if (!plain) {
                 const float* ramp = reinterpret_cast<const float*>(smem + C::kOffRamp);
+                const uint64_t sc2 = pk2(qscale2, qscale2);
 #pragma unroll
-                for (int c = 0; c < 8; ++c) mx8[c] = kNegInf;
-                auto build = [&](auto masked_c) {
-                    constexpr bool kMasked = decltype(masked_c)::value;
+                for (int c4 = 0; c4 < kPK; c4 += 4) {
+                    const float4 b4 = *reinterpret_cast<const float4*>(ramp + c4);
+                    float x[4];
+                    upk2(fma2(pk2(__uint_as_float(sr[c4]), __uint_as_float(sr[c4 + 1])), sc2,
+                              pk2(b4.x, b4.y)),
+                         x[0], x[1]);
+                    upk2(fma2(pk2(__uint_as_float(sr[c4 + 2]), __uint_as_float(sr[c4 + 3])), sc2,
+                              pk2(b4.z, b4.w)),
+                         x[2], x[3]);
 #pragma unroll
-                    for (int c4 = 0; c4 < kPK; c4 += 4) {
-                        const float4 b4 = p.slopes ? *reinterpret_cast<const float4*>(ramp + c4)
-                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
-                        float x[4];
-                        const uint64_t sc2 = pk2(qscale2, qscale2);
-                        upk2(fma2(pk2(__uint_as_float(sr[c4]), __uint_as_float(sr[c4 + 1])), sc2,
-                                  pk2(b4.x, b4.y)),
-                             x[0], x[1]);
-                        upk2(fma2(pk2(__uint_as_float(sr[c4 + 2]), __uint_as_float(sr[c4 + 3])),
-                                  sc2, pk2(b4.z, b4.w)),
-                             x[2], x[3]);
+                    for (int u = 0; u < 4; ++u) sr[c4 + u] = __float_as_uint(x[u]);
+                }
+                if (__any_sync(0xffffffffu, cmax < kPK - 1)) {
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int c = c4 + u;
-                            if (kMasked) x[u] = c <= cmax ? x[u] : kNegInf;
-                            sr[c] = __float_as_uint(x[u]);
-                            mx8[c & 7] = fmaxf(mx8[c & 7], x[u]);
-                        }
-                    }
-                };
-                if (masked)
-                    build(std::true_type{});
-                else
-                    build(std::false_type{});
+                    for (int c = 0; c < kPK; ++c)
+                        if (c > cmax) sr[c] = __float_as_uint(kNegInf);
+                }
             }
-            float mt = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+            float mx8[8];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) mx8[c] = __uint_as_float(sr[c]);
+#pragma unroll
+            for (int k = 1; k < 15; k += 2)
+#pragma unroll
+                for (int c = 0; c < 8; ++c)
+                    mx8[c] = fmax3(mx8[c], __uint_as_float(sr[c + 8 * k]),
+                                   __uint_as_float(sr[c + 8 * (k + 1)]));
+            // columns 120..127 join the final combination
+            float mt = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                             fmax3(mx8[6], mx8[7],
+                                   fmax3(__uint_as_float(sr[120]), __uint_as_float(sr[121]),
+                                         __uint_as_float(sr[122]))));
+            mt = fmax3(mt, fmax3(__uint_as_float(sr[123]), __uint_as_float(sr[124]),
+                                 __uint_as_float(sr[125])),
+                       fmaxf(__uint_as_float(sr[126]), __uint_as_float(sr[127])));
             mt = plain ? mt * qscale2 : mt + ofs;
             // move this row's max when the tile exceeds it by more than the
             // threshold (always on the first tile)
@@ -524,20 +535,18 @@ __global__ void __launch_bounds__(kPThreads, 1)
             // first 64 columns of S_g, and the row sum over independent partials
             // (masked keys give ex2(-inf) = 0)
             uint64_t ls2[2] = {pk2(0.f, 0.f), pk2(0.f, 0.f)};
-            auto exps = [&](auto plain_c) {
-                constexpr bool kPlain = decltype(plain_c)::value;
-                const float mneg = plain ? -m : -(m - ofs);
-                const uint64_t sc2 = pk2(qscale2, qscale2);
-                const uint64_t nm2 = pk2(mneg, mneg);
+            {
+                const float a = plain ? qscale2 : 1.f;
+                const float b = plain ? -m : -(m - ofs);
+                const uint64_t a2 = pk2(a, a), b2 = pk2(b, b);
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     uint32_t w[32];
 #pragma unroll
                     for (int y = 0; y < 32; ++y) {
-                        const float a0 = __uint_as_float(sr[64 * h + 2 * y]);
-                        const float a1 = __uint_as_float(sr[64 * h + 2 * y + 1]);
-                        const uint64_t x = kPlain ? fma2(pk2(a0, a1), sc2, nm2)
-                                                  : add2(pk2(a0, a1), nm2);
+                        const uint64_t x = fma2(pk2(__uint_as_float(sr[64 * h + 2 * y]),
+                                                    __uint_as_float(sr[64 * h + 2 * y + 1])),
+                                                a2, b2);
                         float x0, x1;
                         upk2(x, x0, x1);
                         const float e0 = ex2(x0), e1 = ex2(x1);
@@ -549,11 +558,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
                     }
                     tmem_st32(tmem + lane_addr + s_col + static_cast<uint32_t>(32 * h), w);
                 }
-            };
-            if (plain)
-                exps(std::true_type{});
-            else
-                exps(std::false_type{});
+            }
             {
                 float a0, a1, b0, b1;
                 upk2(ls2[0], a0, a1);

@@ -185,6 +185,8 @@ def test_prefill_rejects_bad_arguments(L):
     assert L.td_prefill(p, p, p, p, p, 1, 1, 0, 128, 1, None, 1, None) == INVALID        # S
     assert L.td_prefill(odd, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID     # align
     assert L.td_prefill(None, p, p, p, p, 1, 1, 64, 128, 1, None, 1, None) == INVALID
+    # key indices are 32-bit in the kernel: S may not come within 256 of 2^31
+    assert L.td_prefill(p, p, p, p, p, 1, 1, 2**31 - 256, 128, 1, None, 1, None) == INVALID
 
 
 def test_wait_test_settings_are_validated(L):
