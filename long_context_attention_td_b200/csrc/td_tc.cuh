@@ -1,6 +1,6 @@
 // td_tc.cuh -- sm_100a tensor-core, TMA and partition helpers shared by the
-// grouped-query kernels (td_gqa.cu: query heads on the MMA M axis;
-// td_gqa_keys.cu: keys on the MMA M axis).
+// tensor-core kernels (td_gqa_keys.cu: grouped-query decode with the keys on
+// the MMA M axis; td_gqa_combine.cu: its merge; td_prefill.cu).
 #pragma once
 
 #include <cuda.h>
